@@ -1,0 +1,436 @@
+"""Benchmark of the online INT8 W8A8 hot path on B200.
+
+Default workload (one "step"): one decode step of the two dense W8A8 linears
+of a Qwen3.6-27B-class MLP at M = 8 tokens -- gate_up (K=5120 -> N=34816) and
+down (K=17408 -> N=5120) -- each a per-token activation quant followed by the
+weight-streaming GEMV with the dequant epilogue.  The headline metric is the
+weight bytes streamed per second.  The same JSON line carries, under "extra",
+the prefill GEMM TOPS (M = 512 / 4096), the routed-MoE layer tokens/s
+(T = 1 / 8 / 512 / 4096) and the FWHT128-domain linear, each with its
+roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--quick]   (headline only, no extra workloads)
+
+Multi-GPU: the path has no exchange step; N ranks run independent replicas
+(weak scaling), timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "W8A8 int8 TOPS (prefill), weight GB/s (decode), MoE layer tokens/s vs roofline"
+
+
+# --------------------------------------------------------------------------- peaks / clocks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------- timing helpers
+def time_events(torch, fn, iters, flush=None):
+    """Mean device time of fn() per call in ms, CUDA events on the current stream,
+    one event pair per call; optional L2 flush between calls (outside the events)."""
+    st = torch.cuda.current_stream()
+    ts = []
+    for _ in range(iters):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(np.mean(ts)), float(np.median(ts))
+
+
+def make_flush(torch, dev):
+    buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        buf.fill_(1)
+    return flush
+
+
+# --------------------------------------------------------------------------- workloads
+def quantize_on_gpu(torch, w8a8, w_np, dev):
+    q, s = w8a8.quant_rows_f32(torch.from_numpy(w_np).to(dev))
+    torch.cuda.synchronize()
+    return q, s
+
+
+def dense_weights(torch, w8a8, inputs, dev, seed=0):
+    rng = np.random.default_rng([seed, 7])
+    out = {}
+    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
+        w = inputs.weights(rng, (d["N"], d["K"]))
+        out[name] = quantize_on_gpu(torch, w8a8, w, dev)
+        del w
+    return out
+
+
+def bf16_dev(torch, bits, dev):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def linear_bytes(M, N, K):
+    """Algorithmic HBM bytes of one W8A8 linear: weights + scales + bf16 in + bf16 out."""
+    return N * K + 4 * N + 2 * M * K + 2 * M * N
+
+
+# --------------------------------------------------------------------------- reference arm (CPU oracle)
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    from moe_gemm_absmax_b200 import inputs
+    oracle.build()
+    cores = oracle.get_threads()
+    M = 8
+    rng = np.random.default_rng([0, 7])
+    rows = {"gate_up": 1024, "down": 256}         # bounded sample of each weight matrix's rows
+    mats = {}
+    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
+        w = inputs.weights(rng, (rows[name], d["K"]))
+        mats[name] = oracle.quant_rows_f32(w)
+    xs = {n: inputs.dense_linear(1, M, d["K"], 16, with_weights=False)[0]
+          for n, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN))}
+    wbytes = sum(mats[n][0].size + 4 * mats[n][0].shape[0] for n in mats)
+
+    def step():
+        for n in mats:
+            oracle.linear(xs[n], *mats[n])
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = wbytes / dt / 1e9
+    sample = (f"decode step at M=8 on the first {rows['gate_up']} of 34816 gate_up rows and "
+              f"{rows['down']} of 5120 down rows; GB/s of those weight bytes")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 scales, bf16 out",
+            "data": "synthetic",
+            "config": {"workload": "decode-shaped dense W8A8 linears, M=8 (gate_up 5120->34816, "
+                                   "down 17408->5120), CPU oracle on a row sample"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+def cpu_baseline(budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the decode workload."""
+    import oracle
+    from moe_gemm_absmax_b200 import inputs
+    oracle.build()
+    rng = np.random.default_rng([0, 7])
+    w = inputs.weights(rng, (2048, inputs.GATE_UP["K"]))
+    qw, sw = oracle.quant_rows_f32(w)
+    xb = inputs.dense_linear(1, 8, inputs.GATE_UP["K"], 16, with_weights=False)[0]
+    oracle.linear(xb, qw, sw)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        oracle.linear(xb, qw, sw)
+        n += 1
+    dt = (time.perf_counter() - t0) / n
+    return {"value": qw.size / dt / 1e9, "unit": "GB/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"gate_up decode linear at M=8 on 2048 of its 34816 weight rows, {n} calls in "
+                      f"{budget_s:.0f} s; GB/s of the sampled int8 weight bytes"}
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, torch, dev):
+    from moe_gemm_absmax_b200 import inputs, w8a8
+    w8a8.lib()       # fails loudly when the CUDA library is missing
+    peaks = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    int8_peak = 2.0 * peaks["bf16_tflops"]           # dense int8 = 2 x dense bf16 (nominal ratio)
+    M = 8
+    W = dense_weights(torch, w8a8, inputs, dev)
+    xs = {}
+    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
+        xs[name] = bf16_dev(torch, inputs.dense_linear(11, M, d["K"], 16, with_weights=False)[0], dev)
+    ys = {n: torch.empty((M, W[n][0].shape[0]), dtype=torch.bfloat16, device=dev) for n in W}
+    wss = {n: torch.empty(max(256, w8a8.linear_workspace_size(M, W[n][0].shape[0], xs[n].shape[1])),
+                          dtype=torch.uint8, device=dev) for n in W}
+    order = ("gate_up", "down")
+
+    def step():
+        for n in order:
+            w8a8.linear(xs[n], W[n][0], W[n][1], y=ys[n], ws=wss[n])
+
+    step_bytes = sum(linear_bytes(M, W[n][0].shape[0], W[n][0].shape[1]) for n in order)
+    weight_bytes = sum(W[n][0].numel() + 4 * W[n][0].shape[0] for n in order)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    with ClockSampler(torch.cuda.current_device() if not os.environ.get("CUDA_VISIBLE_DEVICES") else 0) as clk:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(args.steps):
+            step()
+        e1.record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * weight_bytes / (ms * 1e-3) / 1e9
+
+    # ---- roofline of the dominant kernel: the gate_up GEMV alone (pre-quantized codes)
+    qx, sx = w8a8.quant_act(xs["gate_up"])
+    N, K = W["gate_up"][0].shape
+    y_k = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = make_flush(torch, dev)
+    kfn = lambda: w8a8.gemm_q(qx, sx, W["gate_up"][0], W["gate_up"][1], w8a8.PATH_GEMV, y=y_k)
+    for _ in range(3):
+        kfn()
+    k_ms, k_med = time_events(torch, kfn, 20, flush=flush)
+    k_bytes = N * K + 4 * N + M * K + 4 * M + 2 * M * N
+    achieved = k_bytes / (k_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": None, "kernel": "gemv_dense_kernel<1,8,1> (gate_up, M=8)",
+                "peak_source": peaks["source"] + " (burst copy)"}
+
+    # ---- end to end through the C ABI with host buffers: pinned x in, y out, each step
+    hx = {n: xs[n].cpu().pin_memory() for n in order}
+    hy = {n: torch.empty(ys[n].shape, dtype=torch.bfloat16).pin_memory() for n in order}
+    dx = {n: torch.empty_like(xs[n]) for n in order}
+
+    def e2e_step():
+        for n in order:
+            dx[n].copy_(hx[n], non_blocking=True)
+            w8a8.linear(dx[n], W[n][0], W[n][1], y=ys[n], ws=wss[n])
+            hy[n].copy_(ys[n], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / args.steps
+    h2d = sum(hx[n].numel() * 2 for n in order)
+    d2h = sum(hy[n].numel() * 2 for n in order)
+
+    extra = {} if args.quick else run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush)
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 scales, bf16 in/out", "data": "synthetic",
+            "config": {"workload": "decode-shaped dense W8A8 linears, M=8 tokens: gate_up K=5120->N=34816 then "
+                                   "down K=17408->N=5120 (per-token act quant + weight-streaming GEMV + dequant)",
+                       "tokens": M, "weight_bytes_per_step": weight_bytes, "algorithmic_bytes_per_step": step_bytes,
+                       "l2": "inputs larger than L2: 267 MB of weights streamed per step vs 126 MB L2",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline, "clocks": clk.summary(),
+            "e2e": {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 4 * args.steps, "extra": extra}
+    return line
+
+
+def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
+    out = {}
+    # ---- prefill GEMMs (tcgen05), full linear incl. activation quant
+    for M in (512, 4096):
+        for n in ("gate_up", "down"):
+            N, K = W[n][0].shape
+            x = bf16_dev(torch, inputs.dense_linear(3, M, K, 16, with_weights=False)[0], dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w8a8.linear_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+            qx, sx = w8a8.quant_act(x)
+            fn_lin = lambda: w8a8.linear(x, W[n][0], W[n][1], y=y, ws=ws)
+            fn_gemm = lambda: w8a8.gemm_q(qx, sx, W[n][0], W[n][1], w8a8.PATH_TCGEN05, y=y)
+            for _ in range(3):
+                fn_lin()
+                fn_gemm()
+            t_lin, _ = time_events(torch, fn_lin, 10, flush=flush)
+            t_gemm, _ = time_events(torch, fn_gemm, 10, flush=flush)
+            ops = 2.0 * M * N * K
+            out[f"prefill_{n}_M{M}"] = {
+                "linear_ms": t_lin, "linear_tops": ops / (t_lin * 1e-3) / 1e12,
+                "gemm_ms": t_gemm, "gemm_tops": ops / (t_gemm * 1e-3) / 1e12,
+                "roofline": {"bound": "tensor", "achieved": ops / (t_gemm * 1e-3) / 1e12, "peak": int8_peak,
+                             "unit": "TOPS", "frac": ops / (t_gemm * 1e-3) / 1e12 / int8_peak,
+                             "peak_source": "2 x measured bf16 burst (dense int8 : bf16 = 2 : 1)"}}
+            del x, y, ws, qx, sx
+    # ---- routed MoE layer
+    w13, w2 = inputs.moe_weights(0)
+    q13, s13 = quantize_on_gpu(torch, w8a8, w13, dev)
+    q2, s2 = quantize_on_gpu(torch, w8a8, w2, dev)
+    del w13, w2
+    E, I2, H = q13.shape
+    per_expert = q13[0].numel() + q2[0].numel() + 4 * (I2 + H)
+    for T in (1, 8, 512, 4096):
+        xb, lb = inputs.moe_tokens(0, T)
+        x, lg = bf16_dev(torch, xb, dev), bf16_dev(torch, lb, dev)
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.moe_workspace_size(T, E, H, I2 // 2, 8), dtype=torch.uint8, device=dev)
+        fn = lambda: w8a8.moe_forward(x, lg, q13, s13, q2, s2, 8, y=y, ws=ws)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        _, dbg = w8a8.moe_forward(x, lg, q13, s13, q2, s2, 8, debug=True)
+        touched = int((dbg["counts"] > 0).sum().item())
+        byts = touched * per_expert + 2 * T * H * 2 + 2 * T * E
+        out[f"moe_T{T}"] = {"ms": t, "tokens_per_s": T / (t * 1e-3), "touched_experts": touched,
+                            "roofline": {"bound": "hbm", "achieved": byts / (t * 1e-3) / 1e9, "peak": hbm,
+                                         "unit": "GB/s", "frac": byts / (t * 1e-3) / 1e9 / hbm,
+                                         "bytes": byts}}
+        del x, lg, y, ws
+    del q13, q2
+    # ---- FWHT128-domain linear
+    _, wb = inputs.hadamard_linear(0, 1)
+    qw, sw = w8a8.fwht128_quant(bf16_dev(torch, wb, dev))
+    for M in (1, 2048):
+        xb, _ = inputs.hadamard_linear(M, M)
+        x = bf16_dev(torch, xb, dev)
+        qx, sx = w8a8.fwht128_quant(x)
+        y = torch.empty((M, qw.shape[0]), dtype=torch.bfloat16, device=dev)
+
+        def fn():
+            q, s = w8a8.fwht128_quant(x)
+            w8a8.linear_g128(q, s, qw, sw, y=y)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        N, K = qw.shape
+        ops = 2.0 * M * N * K
+        byts = N * K + 2 * N * (K // 128) + 2 * M * K + 2 * M * N
+        rec = {"ms": t, "tops": ops / (t * 1e-3) / 1e12, "gbs": byts / (t * 1e-3) / 1e9}
+        if M == 1:
+            rec["roofline"] = {"bound": "hbm", "frac": rec["gbs"] / hbm, "peak": hbm, "unit": "GB/s"}
+        else:
+            rec["roofline"] = {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"}
+        out[f"hadamard_M{M}"] = rec
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--quick", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line))
+        return
+
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    line = run_ours(args, rank, world, torch, dev)
+    if rank == 0:
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * w8a8.h -- C ABI of libw8a8.so: online INT8 W8A8 linear layers and the
+ * routed W8A8 MoE expert layer for NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, section):
+ *   [ATOM]  "[gfx1151] Online INT8 W8A8 for Qwen3.6 27B / 35B-A3B on RDNA3.5,
+ *            with working MTP" -- "Precision split" (int8 weights with dynamic
+ *            per-token int8 activations; router gate stays bf16) and "Changes"
+ *            (gemm_a8w8 per-token path; Int8MoEMethod with int8 w13/w2 and
+ *            per-channel fp32 scales; the MoE forward: routing -> per-token int8
+ *            quant -> gemm1 with fused gated SiLU via interleaved w13 -> per-token
+ *            int8 quant -> gemm2 with scatter/combine).
+ *   [QUARK] "Qwen3.6-27B-Quark-W8A8-INT8" -- "Quantization Scheme" and
+ *            "Quantization Details" (per-channel symmetric weights, per-token
+ *            symmetric dynamic activations).
+ *   [IQ8R]  "Qwen3.6-35B-A3B IQ8R - radiance container" -- file table (codes
+ *            -127..127, each 128 of K rotated by the unnormalised Hadamard, a
+ *            bf16 scale per row and 128 of K; activations int8 under the same
+ *            rotation) and the conversion recipe (transform=fwht128 group=128
+ *            scale=bf16 clamp=sym).
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless stated otherwise; the caller owns
+ *     every buffer.  The library allocates nothing, keeps no per-call state
+ *     and never synchronizes: each call enqueues its kernels on `stream`
+ *     (a cudaStream_t; NULL is the legacy default stream) and returns.
+ *   - Matrices are dense and row-major.  bf16 values are passed as their
+ *     16-bit patterns (uint16_t).  Weights are [N, K] with K contiguous.
+ *   - Pointers must be 16-byte aligned; K must be a multiple of 16 (the
+ *     tensor-memory-access unit); N a multiple of 8.
+ *   - Return value: W8A8_OK (0) or a negative W8A8_ERR_* code.  Argument
+ *     errors are detected on the host before anything is enqueued.  A kernel
+ *     that had to give up (a bounded wait ran out) records
+ *     W8A8_ERR_TIMEOUT in a device error word instead of trapping; read it
+ *     with w8a8_get_device_error().
+ */
+#ifndef W8A8_H_
+#define W8A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W8A8_API __attribute__((visibility("default")))
+#else
+#define W8A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W8A8_OK 0
+#define W8A8_ERR_INVALID_ARG (-1)  /* null pointer, bad size, misalignment */
+#define W8A8_ERR_WORKSPACE (-2)    /* workspace smaller than the *_workspace_size query */
+#define W8A8_ERR_UNSUPPORTED (-3)  /* shape outside what the kernels handle */
+#define W8A8_ERR_CUDA (-4)         /* a CUDA launch or driver call failed */
+#define W8A8_ERR_TIMEOUT (-5)      /* a device-side bounded wait gave up */
+
+/* Selects the GEMM kernel in w8a8_gemm_q / w8a8_gemm_s32. */
+#define W8A8_PATH_AUTO 0      /* GEMV for M <= 8 and N % 16 == 0, tensor-core GEMM otherwise */
+#define W8A8_PATH_TCGEN05 1   /* tcgen05 kind::i8 GEMM, any M */
+#define W8A8_PATH_GEMV 2      /* weight-streaming GEMV, M <= 32, N % 16 == 0 */
+
+/* ---------------------------------------------------------------------------
+ * Per-token dynamic activation quantization (a1) -- [ATOM] "Precision split",
+ * [QUARK] "Quantization Scheme" (activation: per-token, symmetric, dynamic).
+ *   x  bf16 [M, K], row stride ldx elements (ldx >= K, ldx % 8 == 0)
+ *   q  int8 [M, K] (row stride K): q = clamp(rne(x / s), -127, 127)
+ *   s  fp32 [M]: s = max_k |x[m,k]| / 127 in fp32; a zero row gives s = 0, q = 0.
+ * Division and rounding are IEEE fp32 round-to-nearest-even. */
+W8A8_API int w8a8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s, void* stream);
+
+/* Online per-output-channel weight quantization (a0) -- [ATOM] "Changes"
+ * (FusedMoE._online_quant; no offline step), [QUARK] "Quantization Scheme"
+ * (weight: per-channel, symmetric).  Same arithmetic as w8a8_quant_act on fp32
+ * rows:  w fp32 [N, K] -> q int8 [N, K], s fp32 [N]. */
+W8A8_API int w8a8_quant_rows_f32(const float* w, int64_t N, int64_t K, int8_t* q, float* s, void* stream);
+
+/* Workspace bytes w8a8_linear needs for an M x K activation. */
+W8A8_API size_t w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* Dense W8A8 linear (a1 + a2 + a3, or a1 + a4 for M <= 8) -- [ATOM] "Changes"
+ * (per-token int8 branch -> gemm_a8w8), [QUARK] "Quantization Details".
+ *   x  bf16 [M, K];  qw int8 [N, K];  sw fp32 [N];  y bf16 [M, N]
+ *   y[m,n] = bf16_rne( (float(sum_k qx[m,k] qw[n,k]) * sx[m]) * sw[n] )
+ * with (qx, sx) = w8a8_quant_act(x) held in `ws` (ws_bytes >=
+ * w8a8_linear_workspace_size(M, N, K)).  The int32 sum is exact. */
+W8A8_API int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* GEMM on pre-quantized activations with the dequant epilogue (a2 + a3):
+ *   qx int8 [M, K], sx fp32 [M], qw int8 [N, K], sw fp32 [N] -> y bf16 [M, N].
+ * `path` is one of W8A8_PATH_*.  The GEMV path with M > 8 and K split over
+ * several CTAs uses `ws` (bytes from w8a8_gemm_workspace_size); pass NULL/0
+ * when w8a8_gemm_workspace_size returns 0. */
+W8A8_API size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int path);
+W8A8_API int w8a8_gemm_q(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, uint16_t* y, int64_t M,
+                int64_t N, int64_t K, int path, void* ws, size_t ws_bytes, void* stream);
+
+/* Raw int32 accumulators (a2), for parity checks:
+ *   acc[m,n] = sum_k qx[m,k] * qw[n,k]   (int32 [M, N], exact). */
+W8A8_API int w8a8_gemm_s32(const int8_t* qx, const int8_t* qw, int32_t* acc, int64_t M, int64_t N, int64_t K, int path,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Routed W8A8 MoE expert layer (a5 .. a11) -- [ATOM] "Changes" (Int8MoEMethod,
+ * triton_kernel_int8_moe_forward), "Precision split" (bf16 router).
+ *   x       bf16 [T, H]             token activations
+ *   logits  bf16 [T, E]             router logits (the bf16 gate GEMM is the caller's)
+ *   w13     int8 [E, 2I, H]         row 2i = gate_i, row 2i+1 = up_i ("interleaved w13")
+ *   s13     fp32 [E, 2I]            per-channel scales of w13
+ *   w2      int8 [E, H, I]; s2 fp32 [E, H]
+ *   y       bf16 [T, H]             output
+ * Steps: top-k of softmax(logits) (ties -> lower expert index), weights
+ * renormalised over the k; x quantized once per token (shared by its
+ * experts); v = (float(qx . w13[e,r]) * sx) * s13[e,r];
+ * a_i = SiLU(v_2i) * v_2i+1; (qa, sa) = per-row quant of a; y2_n =
+ * (float(qa . w2[e,n]) * sa) * s2[e,n]; y = bf16( sum_j w_j * y2 ).  The
+ * combine sums the k contributions in fp32 in an unspecified order.
+ * ws_bytes >= w8a8_moe_workspace_size(T, E, H, I, topk).  `dbg` may be NULL;
+ * otherwise its non-NULL members receive intermediate values. */
+typedef struct w8a8_moe_debug {
+    int32_t* topk_ids;   /* [T, topk], descending logits */
+    float* topk_w;       /* [T, topk] */
+    int32_t* counts;     /* [E] rows routed to each expert */
+    int8_t* qx;          /* [T, H] codes of x */
+    float* sx;           /* [T] */
+    int8_t* qa;          /* [T, topk, I] codes of the gated intermediate, by (token, slot) */
+    float* sa;           /* [T, topk] */
+} w8a8_moe_debug;
+
+W8A8_API size_t w8a8_moe_workspace_size(int64_t T, int E, int H, int I, int topk);
+W8A8_API int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w13, const float* s13,
+                     const int8_t* w2, const float* s2, uint16_t* y, int64_t T, int E, int H, int I, int topk,
+                     void* ws, size_t ws_bytes, const w8a8_moe_debug* dbg, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * FWHT128-domain group quantization (a12) -- [IQ8R] file table ("each 128 of
+ * K rotated by the unnormalised Hadamard"; codes -127..127; a bf16 scale per
+ * row and 128 of K) and recipe (transform=fwht128 group=128 scale=bf16
+ * clamp=sym).  For each 128-wide block of each row of x bf16 [M, K]
+ * (K % 128 == 0): x' = H128 x_blk (unnormalised Sylvester Hadamard, fp32,
+ * butterfly stages 1, 2, 4, ..., 64); s = bf16_rne(max|x'| / 127);
+ * q = clamp(rne(x' / s), -127, 127).
+ *   q int8 [M, K];  s bf16 [M, K/128].
+ * Used for activations at run time and for weights at set-up. */
+W8A8_API int fwht128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, void* stream);
+
+/* Group-128 scaled GEMM in the rotated domain (a13):
+ *   y[m,n] = bf16_rne( (1/128) * sum_g float(p_g) * (sx[m,g] * sw[n,g]) ),
+ *   p_g = sum over the 128 k of group g of qx[m,k] qw[n,k] (int32, exact).
+ * qx int8 [M, K], sx bf16 [M, K/128], qw int8 [N, K], sw bf16 [N, K/128],
+ * y bf16 [M, N].  The fp32 group sum order is unspecified. */
+W8A8_API int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
+                     int64_t M, int64_t N, int64_t K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics. */
+
+/* The library's fp32 exponential (Cody & Waite reduction, degree-7 Taylor),
+ * applied elementwise: y[i] = exp_proj(x[i]).  Used by the router softmax and
+ * by SiLU; exposed so tests can compare it bit for bit. */
+W8A8_API int w8a8_exp_proj(const float* x, float* y, int64_t n, void* stream);
+
+/* Synchronizes `stream`, then returns and clears the device error word:
+ * W8A8_OK or the first W8A8_ERR_* a kernel recorded (W8A8_ERR_CUDA if the
+ * synchronization itself failed).  When site != NULL it receives where the
+ * error was recorded ((kernel id << 16) | site). */
+W8A8_API int w8a8_get_device_error(void* stream, int* site);
+
+/* Test hook for the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing will arrive at, with a limit of `limit_ns` nanoseconds
+ * (1e3 <= limit_ns <= 1e9).  The wait gives up, records W8A8_ERR_TIMEOUT and
+ * the kernel returns; no GPU fault is raised. */
+W8A8_API int w8a8_debug_wait_timeout(int64_t limit_ns, void* stream);
+
+/* Human-readable name of a status code (static string). */
+W8A8_API const char* w8a8_status_str(int status);
+
+/* Library version string (static). */
+W8A8_API const char* w8a8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H_ */

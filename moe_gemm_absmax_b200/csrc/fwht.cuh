@@ -1,0 +1,140 @@
+// FWHT128-domain W8A8 (a12, a13) -- "Qwen3.6-35B-A3B IQ8R - radiance
+// container": file table (each 128 of K rotated by the unnormalised Hadamard;
+// int8 codes -127..127 with a bf16 scale per row and 128 of K; activations
+// int8 under the same rotation) and the recipe (transform=fwht128 group=128
+// scale=bf16 clamp=sym).
+//
+// fwht128_quant_kernel: one warp per 128-wide block of a row.  Lane l holds
+// elements 4l .. 4l+3 in fp32.  The textbook in-place butterflies run stage
+// by stage, h = 1, 2, 4, ..., 64, each pair (a, b) at distance h becoming
+// (a + b, a - b): stages 1 and 2 inside the lane, stages 4 .. 64 between
+// lanes l and l ^ (h / 4) through shuffles.  The same pairs in the same
+// order as the serial loop, so the fp32 result is the same bit for bit.
+// Then s = bf16_rne(max |x'| / 127), q = clamp(rne(x' / float(s)), +-127).
+//
+// gemv_g128_kernel: decode-sized M (<= 8) group-scaled GEMV.  Warps split the
+// K groups, keep each group's exact int32 partial p_g in shared memory, and
+// one warp applies acc = fma(float(p_g), sx*sw, acc) in ascending g -- the
+// same fp32 steps as the serial definition.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace w8a8 {
+
+__global__ void __launch_bounds__(256) fwht128_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
+                                                            int8_t* __restrict__ q, uint16_t* __restrict__ s) {
+    const int lane = threadIdx.x & 31;
+    const int64_t G = K / 128;
+    const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (blk >= M * G) return;
+    const int64_t m = blk / G, g = blk % G;
+    const uint16_t* src = x + m * K + g * 128 + 4 * lane;
+    const uint2 raw = *reinterpret_cast<const uint2*>(src);
+    float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u), __uint_as_float(raw.y << 16),
+                  __uint_as_float(raw.y & 0xffff0000u)};
+    // h = 1: (0,1), (2,3)
+    {
+        const float a0 = v[0], b0 = v[1], a1 = v[2], b1 = v[3];
+        v[0] = __fadd_rn(a0, b0);
+        v[1] = __fsub_rn(a0, b0);
+        v[2] = __fadd_rn(a1, b1);
+        v[3] = __fsub_rn(a1, b1);
+    }
+    // h = 2: (0,2), (1,3)
+    {
+        const float a0 = v[0], b0 = v[2], a1 = v[1], b1 = v[3];
+        v[0] = __fadd_rn(a0, b0);
+        v[2] = __fsub_rn(a0, b0);
+        v[1] = __fadd_rn(a1, b1);
+        v[3] = __fsub_rn(a1, b1);
+    }
+    // h = 4 .. 64: partner lane l ^ (h / 4); the lane with the bit clear holds a
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const bool upper = (lane & d) != 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[j], d);
+            v[j] = upper ? __fsub_rn(o, v[j]) : __fadd_rn(v[j], o);
+        }
+    }
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const uint16_t sb = float_to_bf16_bits(__fdiv_rn(amax, 127.0f));
+    const float sf = bf16_bits_to_float(sb);
+    uint32_t pk = 0u;
+    if (sf != 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pk |= (uint32_t)(uint8_t)(int8_t)quant_code(v[j], sf) << (8 * j);
+    }
+    *reinterpret_cast<uint32_t*>(q + m * K + g * 128 + 4 * lane) = pk;
+    if (lane == 0) s[m * G + g] = sb;
+}
+
+constexpr int kG128MaxGroups = 64;
+
+// One CTA per 16 weight rows; 8 warps split the K groups; tokens <= 8.
+__global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict__ qx,
+                                                        const uint16_t* __restrict__ sx,
+                                                        const int8_t* __restrict__ qw,
+                                                        const uint16_t* __restrict__ sw, uint16_t* __restrict__ y,
+                                                        int M, int N, int K) {
+    __shared__ int4 pg[kG128MaxGroups][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, t = lane & 3;
+    const int G = K / 128;
+    const int block = blockIdx.x;
+    const int8_t* w0 = qw + (int64_t)(block * 16 + g8) * K + 16 * t;
+    const int8_t* w1 = w0 + 8 * (int64_t)K;
+    const bool tok_ok = g8 < M;
+    const int8_t* xr = qx + (int64_t)g8 * K + 16 * t;
+    for (int grp = warp; grp < G; grp += 8) {
+        int acc[4] = {0, 0, 0, 0};
+        uint4 wa[2], wb[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            wa[u] = ld_stream_16(w0 + grp * 128 + u * 64);
+            wb[u] = ld_stream_16(w1 + grp * 128 + u * 64);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            uint4 xb = make_uint4(0, 0, 0, 0);
+            if (tok_ok) xb = __ldg(reinterpret_cast<const uint4*>(xr + grp * 128 + u * 64));
+            const uint32_t A1[4] = {wa[u].x, wb[u].x, wa[u].y, wb[u].y};
+            const uint32_t B1[2] = {xb.x, xb.y};
+            const uint32_t A2[4] = {wa[u].z, wb[u].z, wa[u].w, wb[u].w};
+            const uint32_t B2[2] = {xb.z, xb.w};
+            mma_s8_16832(acc, A1, B1);
+            mma_s8_16832(acc, A2, B2);
+        }
+        pg[grp][lane] = make_int4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    float yv[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int grp = 0; grp < G; ++grp) {
+        const int4 p = pg[grp][lane];
+        const int pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int m = 2 * t + (j & 1);
+            const int n = block * 16 + g8 + 8 * (j >> 1);
+            if (m < M) {
+                const float sc = __fmul_rn(bf16_bits_to_float(__ldg(sx + (int64_t)m * G + grp)),
+                                           bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp)));
+                yv[j] = __fmaf_rn(__int2float_rn(pv[j]), sc, yv[j]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int m = 2 * t + (j & 1);
+        const int n = block * 16 + g8 + 8 * (j >> 1);
+        if (m < M && n < N) y[(int64_t)m * N + n] = float_to_bf16_bits(__fmul_rn(yv[j], 0.0078125f));
+    }
+}
+
+}  // namespace w8a8

@@ -1,0 +1,321 @@
+// int8 x int8 -> int32 GEMMs on the 5th-generation tensor cores.
+//
+// (a2 + a3) dense W8A8 -- "Online INT8 W8A8 ...", Changes (gemm_a8w8
+// per-token path); "Qwen3.6-27B-Quark-W8A8-INT8", Quantization Details:
+//   acc[m,n] = sum_k A[m,k] B[n,k]                      A = codes [M,K], B = weights [N,K]
+//   y[m,n]   = bf16_rne( (float(acc) * sx[m]) * sw[n] )  (or the raw int32 acc)
+// (a13) group-128 scaled, rotated domain -- "Qwen3.6-35B-A3B IQ8R - radiance
+// container", file table (a bf16 scale per row and 128 of K):
+//   p_g      = sum over the 128 k of group g of A[m,k] B[n,k]   (one TMEM tile per g)
+//   acc      = fma(float(p_g), float(sx[m,g]) * float(sw[n,g]), acc), g ascending
+//   y[m,n]   = bf16_rne(acc * (1/128))
+//
+// Persistent, warp-specialised CTA (one per SM, 192 threads):
+//   warp 0      TMA producer: 128-byte-swizzled K-major tiles of A (128 x 128)
+//               and B (BN x 128) into a STAGES-deep shared-memory ring;
+//   warp 1      TMEM allocator and single-thread tcgen05.mma.kind::i8 issuer
+//               (M=128, N=BN, K=32 per instruction) into NACC rotating TMEM
+//               accumulators, so the epilogue overlaps the next MMAs;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane TMEM quarter, dequant
+//               (or per-group promotion), bf16 pack, 16-byte global stores.
+// A dense tile hands its accumulator to the epilogue once, after the whole
+// K loop; a group-128 tile hands over one accumulator per 128-wide k block.
+// Every wait is bounded (mbar_wait_bounded); a CTA that gives up drains its
+// own copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include "common.cuh"
+
+namespace w8a8 {
+
+constexpr int kTcBM = 128;
+constexpr int kTcBK = 128;          // int8 elements (= bytes) of K per stage: one swizzle atom
+constexpr int kTcThreads = 192;
+constexpr int kKernelIdGemmTc = 1;
+
+enum TcEpilogue : int { kEpiBf16 = 0, kEpiS32 = 1, kEpiG128 = 2 };
+
+struct TcParams {
+    int M, N, K;
+    int num_m_tiles, num_n_tiles, num_k_blocks;
+    const float* sx;        // [M]        (kEpiBf16)
+    const float* sw;        // [N]        (kEpiBf16)
+    const uint16_t* gsx;    // [M, G] bf16 (kEpiG128)
+    const uint16_t* gsw;    // [N, G] bf16 (kEpiG128)
+    void* out;              // bf16 or int32 [M, N], row stride N
+};
+
+template <int BN, int STAGES>
+struct TcSmem {
+    static constexpr int kA = kTcBM * kTcBK;                 // bytes per A stage
+    static constexpr int kB = BN * kTcBK;                    // bytes per B stage
+    static constexpr int kTiles = STAGES * (kA + kB);
+    static constexpr int kBars = (2 * STAGES + 2 * 4 + 1) * 8;
+    static constexpr int kBytes = 1024 /*alignment slack*/ + kTiles + kBars + 16;
+};
+
+template <int BN, int STAGES, int EPI, int NACC>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    static_assert(NACC >= 2 && NACC <= 4, "NACC");
+    constexpr int kCols = NACC * BN;
+    static_assert(kCols == 64 || kCols == 128 || kCols == 256 || kCols == 512, "TMEM columns: power of two");
+    static_assert(EPI != kEpiG128 || BN <= 128, "group-128 epilogue keeps BN fp32 sums per thread");
+    using SM = TcSmem<BN, STAGES>;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * SM::kA;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kTiles);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = tfull + 4;
+    uint64_t* mma_done = tempty + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < NACC; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0;          // bit s: stage s was loaded at least once
+            uint32_t last_phase = 0;      // bit s: phase of the last load into stage s
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int mt = tile % p.num_m_tiles;
+                const int nt = tile / p.num_m_tiles;
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, (kKernelIdGemmTc << 16) | 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(SM::kA + SM::kB));
+                    tma_load_2d(sA + stage * SM::kA, &tmA, &full[stage], kb * kTcBK, mt * kTcBM);
+                    tma_load_2d(sB + stage * SM::kB, &tmB, &full[stage], kb * kTcBK, nt * BN);
+                    issued |= 1u << stage;
+                    last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: every copy this thread started lands before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait_bounded(&full[s], (last_phase >> s) & 1u, nullptr, (kKernelIdGemmTc << 16) | 2,
+                                          100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(kTcBM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                    const bool new_acc = (EPI == kEpiG128) || kb == 0;
+                    if (new_acc) {
+                        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag,
+                                               (kKernelIdGemmTc << 16) | 3)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, (kKernelIdGemmTc << 16) | 4)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                    const uint32_t a0 = smem_u32(sA + stage * SM::kA);
+                    const uint32_t b0 = smem_u32(sB + stage * SM::kB);
+#pragma unroll
+                    for (int kk = 0; kk < kTcBK / 32; ++kk) {
+                        const bool accumulate = kk > 0 || (EPI != kEpiG128 && kb > 0);
+                        tc_mma_i8(d_tmem, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
+                                  accumulate ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);       // frees the smem stage when these MMAs finish
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    const bool hand_over = (EPI == kEpiG128) || kb == p.num_k_blocks - 1;
+                    if (hand_over) {
+                        tc_commit(&tfull[acc]);     // accumulator ready for the epilogue
+                        if (++acc == NACC) {
+                            acc = 0;
+                            acc_phase ^= 1u;
+                        }
+                    }
+                }
+            }
+            // all MMAs issued by this thread complete before TMEM is released
+            tc_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0u, nullptr, (kKernelIdGemmTc << 16) | 5, 100000000ull);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;                 // TMEM lanes [32 q, 32 q + 32)
+        const int row_in_tile = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            const int mt = tile % p.num_m_tiles;
+            const int nt = tile / p.num_m_tiles;
+            const int row = mt * kTcBM + row_in_tile;
+            const bool row_ok = row < p.M;
+            const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
+            if constexpr (EPI == kEpiG128) {
+                const int G = p.num_k_blocks;
+                float y[BN];
+#pragma unroll
+                for (int j = 0; j < BN; ++j) y[j] = 0.0f;
+                for (int kb = 0; kb < G; ++kb) {
+                    if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float sxg = row_ok ? bf16_bits_to_float(__ldg(p.gsx + (int64_t)row * G + kb)) : 0.0f;
+#pragma unroll
+                    for (int c = 0; c < BN; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tq + (uint32_t)(acc * BN + c), r);
+                        // lane i fetches the weight scale of column n0 + i; shuffles share it
+                        const int ncol = nt * BN + c + lane;
+                        const float swl =
+                            ncol < p.N ? bf16_bits_to_float(__ldg(p.gsw + (int64_t)ncol * G + kb)) : 0.0f;
+                        tc_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float sc = __fmul_rn(sxg, __shfl_sync(0xffffffffu, swl, j));
+                            y[c + j] = __fmaf_rn(__int2float_rn((int)r[j]), sc, y[c + j]);
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&tempty[acc]);
+                    if (++acc == NACC) {
+                        acc = 0;
+                        acc_phase ^= 1u;
+                    }
+                }
+                if (ok && row_ok) {
+                    uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
+#pragma unroll
+                    for (int v = 0; v < BN / 8; ++v) {
+                        const int n0 = nt * BN + v * 8;
+                        if (n0 < p.N) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                pk[j] = pack_bf16x2(__fmul_rn(y[v * 8 + 2 * j], 0.0078125f),
+                                                    __fmul_rn(y[v * 8 + 2 * j + 1], 0.0078125f));
+                            *reinterpret_cast<uint4*>(yrow + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+            } else {
+                if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) break;
+                tc_fence_after();
+                float sxr = 0.0f;
+                if (EPI == kEpiBf16 && row_ok) sxr = __ldg(p.sx + row);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tq + (uint32_t)(acc * BN + c), r);
+                    tc_wait_ld();
+                    const int n0 = nt * BN + c;
+                    if (!row_ok || n0 >= p.N) continue;
+                    if (EPI == kEpiBf16) {
+                        uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
+                        const float4* swv = reinterpret_cast<const float4*>(p.sw + n0);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {           // 8 columns per 16-byte store
+                            if (n0 + v * 8 < p.N) {
+                                const float4 s0 = __ldg(swv + 2 * v);
+                                const float4 s1 = __ldg(swv + 2 * v + 1);
+                                const float sw8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                                uint32_t pk[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const float lo = __fmul_rn(
+                                        __fmul_rn(__int2float_rn((int)r[v * 8 + 2 * j]), sxr), sw8[2 * j]);
+                                    const float hi = __fmul_rn(
+                                        __fmul_rn(__int2float_rn((int)r[v * 8 + 2 * j + 1]), sxr), sw8[2 * j + 1]);
+                                    pk[j] = pack_bf16x2(lo, hi);
+                                }
+                                *reinterpret_cast<uint4*>(yrow + n0 + v * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            }
+                        }
+                    } else {
+                        int32_t* orow = reinterpret_cast<int32_t*>(p.out) + (int64_t)row * p.N;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            if (n0 + v * 4 < p.N)
+                                *reinterpret_cast<uint4*>(orow + n0 + v * 4) =
+                                    make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+                if (++acc == NACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kCols);
+    }
+}
+
+}  // namespace w8a8

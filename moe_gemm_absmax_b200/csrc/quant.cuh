@@ -1,0 +1,182 @@
+// Per-row symmetric absmax int8 quantization (a0 weights, a1 activations,
+// a9 MoE requant) -- "Qwen3.6-27B-Quark-W8A8-INT8", Quantization Scheme
+// (per-channel / per-token symmetric); "Online INT8 W8A8 ...", Precision
+// split (dynamic per-token int8 activation).
+//
+//   s = max_k |v_k| / 127           (fp32, IEEE division)
+//   q = clamp(rne(v_k / s), -127, 127),  s == 0 -> q = 0
+//
+// One pass over HBM: each CTA keeps its slice of the row in registers
+// (16-byte vector loads), reduces |v| with warp shuffles, and for short
+// rows (decode: few tokens, long K) a thread-block cluster splits one row
+// over up to 8 CTAs whose partial maxima meet through distributed shared
+// memory.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace w8a8 {
+
+namespace cg = cooperative_groups;
+
+constexpr int kQuantMaxVec = 16;   // 16-byte vectors kept in registers per thread
+
+template <typename Tin>
+struct VecTraits;
+template <>
+struct VecTraits<uint16_t> {   // bf16 bits: 8 per 16 bytes
+    static constexpr int kElems = 8;
+    __device__ static void unpack(const uint4& v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+template <>
+struct VecTraits<float> {      // fp32: 4 per 16 bytes
+    static constexpr int kElems = 4;
+    __device__ static void unpack(const uint4& v, float (&f)[4]) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// grid = (CL * rows); cluster = (CL, 1, 1).  Cluster r handles row r; its
+// CTA c handles vectors [c * vpc, (c + 1) * vpc) (vpc = vectors per CTA).
+template <typename Tin, int NT>
+__global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ x, int64_t K, int64_t ldx,
+                                                        int8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
+                                                        int vpc, int cl, int* zero_buf, int zero_n) {
+    using VT = VecTraits<Tin>;
+    // optional side job: clear a small int buffer that a later kernel on the
+    // same stream expects to find zero (split-K arrival counters)
+    for (int i = blockIdx.x * NT + threadIdx.x; i < zero_n; i += gridDim.x * NT) zero_buf[i] = 0;
+    constexpr int E = VT::kElems;
+    const int64_t row = blockIdx.x / cl;
+    const int crank = blockIdx.x % cl;
+    const int64_t nvec = K / E;
+    const int64_t v0 = (int64_t)crank * vpc;
+    const int64_t v1 = min(nvec, v0 + vpc);
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
+
+    uint4 regs[kQuantMaxVec];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kQuantMaxVec; ++i) {
+        const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
+        if (v < v1) {
+            regs[i] = __ldg(xr + v);
+            float f[E];
+            VT::unpack(regs[i], f);
+#pragma unroll
+            for (int j = 0; j < E; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        }
+    }
+    __shared__ float red[NT / 32];
+    __shared__ float cta_max;
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = red[0];
+#pragma unroll
+        for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, red[w]);
+        cta_max = m;
+    }
+    if (cl > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        if (threadIdx.x == 0) {
+            float m = 0.0f;
+            for (int r = 0; r < cl; ++r) m = fmaxf(m, *cluster.map_shared_rank(&cta_max, r));
+            red[0] = m;
+        }
+        cluster.sync();   // no CTA leaves while a peer may still read its cta_max
+    } else {
+        __syncthreads();
+        if (threadIdx.x == 0) red[0] = cta_max;
+    }
+    __syncthreads();
+    amax = red[0];
+    const float sc = __fdiv_rn(amax, 127.0f);
+    if (crank == 0 && threadIdx.x == 0) s[row] = sc;
+
+    int8_t* qr = q + row * ldq;
+#pragma unroll
+    for (int i = 0; i < kQuantMaxVec; ++i) {
+        const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
+        if (v < v1) {
+            float f[E];
+            VT::unpack(regs[i], f);
+            uint32_t packed[E / 4];
+#pragma unroll
+            for (int j = 0; j < E / 4; ++j) packed[j] = 0u;
+            if (sc != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < E; ++j) {
+                    const uint32_t b = (uint32_t)(uint8_t)(int8_t)quant_code(f[j], sc);
+                    packed[j >> 2] |= b << (8 * (j & 3));
+                }
+            }
+            if constexpr (E == 8) {
+                *reinterpret_cast<uint2*>(qr + v * E) = make_uint2(packed[0], packed[1]);
+            } else {
+                *reinterpret_cast<uint32_t*>(qr + v * E) = packed[0];
+            }
+        }
+    }
+}
+
+// Picks the cluster width and launches.  Requirements (checked by callers):
+// K % (16 / sizeof(Tin)) == 0, ldx likewise, 16-byte aligned x, 8-byte aligned q rows.
+template <typename Tin>
+cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* s,
+                              cudaStream_t stream, int num_sms, int* zero_buf = nullptr, int zero_n = 0) {
+    constexpr int E = VecTraits<Tin>::kElems;
+    const int64_t nvec = K / E;
+    int NT = nvec <= 64 ? 64 : (nvec <= 128 ? 128 : 256);
+    // smallest cluster width that fits the row in registers
+    int cl = (int)((nvec + (int64_t)NT * kQuantMaxVec - 1) / ((int64_t)NT * kQuantMaxVec));
+    if (cl < 1) cl = 1;
+    // few rows: widen the cluster so that more SMs pull the row from HBM
+    while (cl < 8 && rows * cl < 2 * num_sms && nvec / (cl * 2) >= (int64_t)NT) cl *= 2;
+    if (cl > 8) return cudaErrorInvalidValue;
+    int vpc = (int)((nvec + cl - 1) / cl);
+
+    cudaLaunchConfig_t cfg = {};
+    if (rows * cl > 0x7fffffffLL) return cudaErrorInvalidValue;
+    cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
+    cfg.blockDim = dim3((unsigned)NT, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    switch (NT) {
+        case 64:
+            return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, 64>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n);
+        case 128:
+            return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, 128>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n);
+        default:
+            return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, 256>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n);
+    }
+}
+
+}  // namespace w8a8

@@ -1,0 +1,561 @@
+// libw8a8.so: the C ABI declared in include/w8a8.h.
+//
+// Host side only: argument checks, workspace carving, kernel selection and
+// launches.  Every entry point enqueues on the caller's stream, allocates
+// nothing and never synchronizes (w8a8_get_device_error excepted, which is
+// documented to synchronize).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "fwht.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "moe.cuh"
+#include "quant.cuh"
+#include "w8a8.h"
+
+using namespace w8a8;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int device_sms(int dev) {
+    static int sms[kMaxDevices] = {0};
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    if (sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        sms[dev] = v;
+    }
+    return sms[dev];
+}
+
+int current_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    return device_sms(dev);
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA; }
+
+inline int last_launch_status() { return cuda_status(cudaGetLastError()); }
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ----------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// int8 matrix [rows, cols] (row stride cols bytes) read as box_rows x 128-byte tiles, 128-byte swizzle.
+bool make_tmap_i8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols};
+    cuuint32_t box[2] = {(cuuint32_t)kTcBK, box_rows};
+    cuuint32_t estride[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- tcgen05 GEMM
+template <int BN, int STAGES, int EPI, int NACC>
+int launch_tc(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
+    using SM = TcSmem<BN, STAGES>;
+    auto kern = gemm_i8_tc_kernel<BN, STAGES, EPI, NACC>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    static bool attr_done[kMaxDevices] = {false};
+    if (dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    CUtensorMap ta, tb;
+    if (!make_tmap_i8(&ta, A, (uint64_t)p.M, (uint64_t)p.K, kTcBM)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tb, B, (uint64_t)p.N, (uint64_t)p.K, BN)) return W8A8_ERR_CUDA;
+    p.num_m_tiles = (p.M + kTcBM - 1) / kTcBM;
+    p.num_n_tiles = (p.N + BN - 1) / BN;
+    p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
+    const int tiles = p.num_m_tiles * p.num_n_tiles;
+    const int grid = tiles < device_sms(dev) ? tiles : device_sms(dev);
+    kern<<<grid, kTcThreads, SM::kBytes, st>>>(ta, tb, p);
+    return last_launch_status();
+}
+
+// Tile width: the one with less work in its last wave (256 on ties).
+int pick_bn(int64_t M, int64_t N, int sms) {
+    const int64_t mt = (M + kTcBM - 1) / kTcBM;
+    const int64_t w256 = (mt * ((N + 255) / 256) + sms - 1) / sms;
+    const int64_t w128 = (mt * ((N + 127) / 128) + sms - 1) / sms;
+    return (w128 * 128 < w256 * 256) ? 128 : 256;
+}
+
+int run_tc(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M, int64_t N,
+           int64_t K, int epi, cudaStream_t st) {
+    TcParams p = {};
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.sx = sx;
+    p.sw = sw;
+    p.out = out;
+    const int bn = pick_bn(M, N, current_sms());
+    if (epi == kEpiBf16)
+        return bn == 256 ? launch_tc<256, 4, kEpiBf16, 2>(qx, qw, p, st) : launch_tc<128, 6, kEpiBf16, 2>(qx, qw, p, st);
+    return bn == 256 ? launch_tc<256, 4, kEpiS32, 2>(qx, qw, p, st) : launch_tc<128, 6, kEpiS32, 2>(qx, qw, p, st);
+}
+
+// ----------------------------------------------------------------- GEMV
+struct GemvPlan {
+    int wn, wk, tg, nkseg;
+    int ctas_x;        // CTAs along the rows
+};
+
+// Fixed for a shape (independent of the device) so that workspace sizes are too.
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
+    GemvPlan g;
+    g.tg = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+    g.wn = 1;
+    g.wk = 8;
+    const int64_t nchunks = (K + 63) / 64;
+    if (nchunks < 16) {          // short K: warps take separate row blocks
+        g.wn = 8;
+        g.wk = 1;
+    }
+    const int64_t blocks = (N + 15) / 16;
+    g.ctas_x = (int)((blocks + g.wn - 1) / g.wn);
+    const int64_t target = 148 * 8;   // ~8 resident CTAs per SM over the 148 SMs of a B200
+    int s = 1;
+    while (s < 8 && (int64_t)g.ctas_x * s * 2 <= target + target / 2 && nchunks / (g.wk * s * 2) >= 2) s *= 2;
+    g.nkseg = s;
+    return g;
+}
+
+size_t gemv_ws_bytes(const GemvPlan& g, int64_t N) {
+    if (g.nkseg == 1) return 0;
+    const int64_t blocks = (N + 15) / 16;
+    return align_up((size_t)g.nkseg * blocks * g.tg * 32 * 16, 256) + align_up((size_t)g.ctas_x * 4, 256);
+}
+
+template <int WN, int WK, int TG>
+int launch_gemv_t(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g, cudaStream_t st) {
+    dim3 grid((unsigned)g.ctas_x, (unsigned)g.nkseg, 1);
+    gemv_dense_kernel<WN, WK, TG><<<grid, kGemvThreads, 0, st>>>(a, e);
+    return last_launch_status();
+}
+
+int launch_gemv(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g, cudaStream_t st) {
+    if (g.wn == 1) {
+        if (g.tg == 1) return launch_gemv_t<1, 8, 1>(a, e, g, st);
+        if (g.tg == 2) return launch_gemv_t<1, 8, 2>(a, e, g, st);
+        return launch_gemv_t<1, 8, 4>(a, e, g, st);
+    }
+    if (g.tg == 1) return launch_gemv_t<8, 1, 1>(a, e, g, st);
+    if (g.tg == 2) return launch_gemv_t<8, 1, 2>(a, e, g, st);
+    return launch_gemv_t<8, 1, 4>(a, e, g, st);
+}
+
+// Runs the GEMV given the split-K scratch (counters must be zero on entry).
+int run_gemv(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M, int64_t N,
+             int64_t K, bool s32, const GemvPlan& g, void* scratch, cudaStream_t st) {
+    GemvShape a;
+    a.w = qw;
+    a.x = qx;
+    a.tokens = (int)M;
+    a.rows = (int)N;
+    a.K = (int)K;
+    a.nchunks = (int)((K + 63) / 64);
+    a.part = nullptr;
+    a.counters = nullptr;
+    if (g.nkseg > 1) {
+        const int64_t blocks = (N + 15) / 16;
+        a.part = reinterpret_cast<int32_t*>(scratch);
+        a.counters = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(scratch) +
+                                            align_up((size_t)g.nkseg * blocks * g.tg * 32 * 16, 256));
+    }
+    GemvEpiDense e;
+    e.sx = sx;
+    e.sw = sw;
+    e.out = out;
+    e.M = (int)M;
+    e.N = (int)N;
+    e.s32 = s32 ? 1 : 0;
+    return launch_gemv(a, e, g, st);
+}
+
+int* gemv_counters(const GemvPlan& g, int64_t N, void* scratch) {
+    if (g.nkseg == 1) return nullptr;
+    const int64_t blocks = (N + 15) / 16;
+    return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(scratch) +
+                                  align_up((size_t)g.nkseg * blocks * g.tg * 32 * 16, 256));
+}
+
+bool gemm_shape_ok(int64_t M, int64_t N, int64_t K) {
+    return M > 0 && N > 0 && K > 0 && K % 16 == 0 && N % 8 == 0 && M <= (1 << 30) && N <= (1 << 30) &&
+           K <= (1 << 30);
+}
+
+// ----------------------------------------------------------------- misc kernels
+__global__ void exp_proj_kernel(const float* x, float* y, int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = exp_proj(x[i]);
+}
+
+constexpr int kKernelIdDebugWait = 9;
+
+__global__ void debug_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);   // one arrival expected; nobody arrives
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    mbar_wait_bounded(&bar, 0u, &abort_flag, (kKernelIdDebugWait << 16) | 1, limit_ns);
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------- MoE
+namespace {
+struct MoeWs {
+    int32_t* ids;
+    float* wts;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* active;
+    int32_t* n_active;
+    int32_t* row_of;
+    int32_t* row_tok;
+    int32_t* row_slot;
+    float* row_w;
+    int8_t* xq;
+    float* sxr;
+    float* a;
+    int8_t* qa;
+    float* sa;
+    float* out;
+    size_t bytes;
+};
+
+MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
+    MoeWs w;
+    const int64_t R = T * topk;
+    uint8_t* p = reinterpret_cast<uint8_t*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* r = p ? p + o : nullptr;
+        o += align_up(bytes, 256);
+        return r;
+    };
+    w.ids = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.wts = reinterpret_cast<float*>(take((size_t)R * 4));
+    w.counts = reinterpret_cast<int32_t*>(take((size_t)E * 4));
+    w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+    w.active = reinterpret_cast<int32_t*>(take((size_t)E * 4));
+    w.n_active = reinterpret_cast<int32_t*>(take(4));
+    w.row_of = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_tok = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_slot = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_w = reinterpret_cast<float*>(take((size_t)R * 4));
+    w.xq = reinterpret_cast<int8_t*>(take((size_t)R * H));
+    w.sxr = reinterpret_cast<float*>(take((size_t)R * 4));
+    w.a = reinterpret_cast<float*>(take((size_t)R * I * 4));
+    w.qa = reinterpret_cast<int8_t*>(take((size_t)R * I));
+    w.sa = reinterpret_cast<float*>(take((size_t)R * 4));
+    w.out = reinterpret_cast<float*>(take((size_t)T * H * 4));
+    w.bytes = o;
+    return w;
+}
+
+template <int WN, int WK, int TG, bool GATED>
+int launch_moe_gemm(const MoeGemmArgs& m, int ctas_x, int max_active, cudaStream_t st) {
+    dim3 grid((unsigned)ctas_x, (unsigned)max_active, 1);
+    moe_gemm_kernel<WN, WK, TG, GATED><<<grid, kGemvThreads, 0, st>>>(m);
+    return last_launch_status();
+}
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char* w8a8_version(void) { return "w8a8 sm_100a 0.1"; }
+
+const char* w8a8_status_str(int status) {
+    switch (status) {
+        case W8A8_OK:
+            return "ok";
+        case W8A8_ERR_INVALID_ARG:
+            return "invalid argument";
+        case W8A8_ERR_WORKSPACE:
+            return "workspace too small";
+        case W8A8_ERR_UNSUPPORTED:
+            return "unsupported shape";
+        case W8A8_ERR_CUDA:
+            return "CUDA error";
+        case W8A8_ERR_TIMEOUT:
+            return "device wait timed out";
+        default:
+            return "unknown status";
+    }
+}
+
+int w8a8_quant_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s, void* stream) {
+    if (!x || !q || !s || M <= 0 || K <= 0 || K % 16 != 0 || ldx < K || ldx % 8 != 0) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return W8A8_ERR_INVALID_ARG;
+    if (K / 8 > (int64_t)8 * 256 * kQuantMaxVec) return W8A8_ERR_UNSUPPORTED;
+    cudaError_t e = launch_quant_rows<uint16_t>(x, M, K, ldx, q, K, s, (cudaStream_t)stream, current_sms());
+    return cuda_status(e);
+}
+
+int w8a8_quant_rows_f32(const float* w, int64_t N, int64_t K, int8_t* q, float* s, void* stream) {
+    if (!w || !q || !s || N <= 0 || K <= 0 || K % 16 != 0) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(q, 16) || !aligned(s, 4)) return W8A8_ERR_INVALID_ARG;
+    if (K / 4 > (int64_t)8 * 256 * kQuantMaxVec) return W8A8_ERR_UNSUPPORTED;
+    cudaError_t e = launch_quant_rows<float>(w, N, K, K, q, K, s, (cudaStream_t)stream, current_sms());
+    return cuda_status(e);
+}
+
+size_t w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    size_t b = align_up((size_t)M * K, 256) + align_up((size_t)M * 4, 256);
+    if (M <= 8 && N % 16 == 0) b += gemv_ws_bytes(gemv_plan(M, N, K), N);
+    return b;
+}
+
+int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !qw || !sw || !y || !ws) return W8A8_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(M, N, K)) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(qw, 16) || !aligned(sw, 16) || !aligned(y, 16) || !aligned(ws, 256))
+        return W8A8_ERR_INVALID_ARG;
+    if (ws_bytes < w8a8_linear_workspace_size(M, N, K)) return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    int8_t* qx = reinterpret_cast<int8_t*>(ws);
+    float* sx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + align_up((size_t)M * K, 256));
+    void* scratch = reinterpret_cast<uint8_t*>(sx) + align_up((size_t)M * 4, 256);
+    const bool gemv = M <= 8 && N % 16 == 0;
+    GemvPlan g = gemv_plan(M, N, K);
+    int* ctr = gemv ? gemv_counters(g, N, scratch) : nullptr;
+    if (K / 8 > (int64_t)8 * 256 * kQuantMaxVec) return W8A8_ERR_UNSUPPORTED;
+    cudaError_t e = launch_quant_rows<uint16_t>(x, M, K, K, qx, K, sx, st, current_sms(), ctr, ctr ? g.ctas_x : 0);
+    if (e != cudaSuccess) return W8A8_ERR_CUDA;
+    if (gemv) return run_gemv(qx, sx, qw, sw, y, M, N, K, false, g, scratch, st);
+    return run_tc(qx, sx, qw, sw, y, M, N, K, kEpiBf16, st);
+}
+
+size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int path) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8 && N % 16 == 0);
+    if (!gemv) return 0;
+    return gemv_ws_bytes(gemv_plan(M, N, K), N);
+}
+
+static int gemm_common(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M,
+                       int64_t N, int64_t K, int path, void* ws, size_t ws_bytes, bool s32, cudaStream_t st) {
+    if (!qx || !qw || !out) return W8A8_ERR_INVALID_ARG;
+    if (!s32 && (!sx || !sw)) return W8A8_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(M, N, K)) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(out, 16)) return W8A8_ERR_INVALID_ARG;
+    if (!s32 && (!aligned(sx, 4) || !aligned(sw, 16))) return W8A8_ERR_INVALID_ARG;
+    if (path < W8A8_PATH_AUTO || path > W8A8_PATH_GEMV) return W8A8_ERR_INVALID_ARG;
+    const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8 && N % 16 == 0);
+    if (gemv) {
+        if (M > 32 || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
+        GemvPlan g = gemv_plan(M, N, K);
+        const size_t need = gemv_ws_bytes(g, N);
+        if (need > 0) {
+            if (!ws || !aligned(ws, 256)) return W8A8_ERR_INVALID_ARG;
+            if (ws_bytes < need) return W8A8_ERR_WORKSPACE;
+            if (cudaMemsetAsync(gemv_counters(g, N, ws), 0, (size_t)g.ctas_x * 4, st) != cudaSuccess)
+                return W8A8_ERR_CUDA;
+        }
+        return run_gemv(qx, sx, qw, sw, out, M, N, K, s32, g, ws, st);
+    }
+    return run_tc(qx, sx, qw, sw, out, M, N, K, s32 ? kEpiS32 : kEpiBf16, st);
+}
+
+int w8a8_gemm_q(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, uint16_t* y, int64_t M,
+                int64_t N, int64_t K, int path, void* ws, size_t ws_bytes, void* stream) {
+    return gemm_common(qx, sx, qw, sw, y, M, N, K, path, ws, ws_bytes, false, (cudaStream_t)stream);
+}
+
+int w8a8_gemm_s32(const int8_t* qx, const int8_t* qw, int32_t* acc, int64_t M, int64_t N, int64_t K, int path,
+                  void* ws, size_t ws_bytes, void* stream) {
+    return gemm_common(qx, nullptr, qw, nullptr, acc, M, N, K, path, ws, ws_bytes, true, (cudaStream_t)stream);
+}
+
+
+size_t w8a8_moe_workspace_size(int64_t T, int E, int H, int I, int topk) {
+    if (T <= 0 || E <= 0 || H <= 0 || I <= 0 || topk <= 0) return 0;
+    return moe_carve(nullptr, T, E, H, I, topk).bytes;
+}
+
+int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w13, const float* s13,
+                     const int8_t* w2, const float* s2, uint16_t* y, int64_t T, int E, int H, int I, int topk,
+                     void* ws, size_t ws_bytes, const w8a8_moe_debug* dbg, void* stream) {
+    if (!x || !logits || !w13 || !s13 || !w2 || !s2 || !y || !ws) return W8A8_ERR_INVALID_ARG;
+    if (T <= 0 || E <= 0 || H <= 0 || I <= 0 || topk <= 0 || topk > E || topk > kMoeMaxTopk) return W8A8_ERR_INVALID_ARG;
+    if (E > 256) return W8A8_ERR_UNSUPPORTED;
+    if (H % 64 != 0 || I % 64 != 0 || H > 8192 || I > 8192) return W8A8_ERR_UNSUPPORTED;
+    if (T * topk > (int64_t)1 << 30 || T > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(logits, 2) || !aligned(w13, 16) || !aligned(s13, 4) || !aligned(w2, 16) ||
+        !aligned(s2, 4) || !aligned(y, 16) || !aligned(ws, 256))
+        return W8A8_ERR_INVALID_ARG;
+    if (ws_bytes < w8a8_moe_workspace_size(T, E, H, I, topk)) return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    MoeWs w = moe_carve(ws, T, E, H, I, topk);
+    const int64_t R = T * topk;
+    int rc;
+
+    moe_route_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts);
+    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+
+    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.row_of, w.row_tok, w.row_slot, w.row_w};
+    moe_plan_kernel<<<1, 1024, 0, st>>>(w.ids, w.wts, R, E, topk, plan);
+    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+
+    moe_quant_scatter_kernel<<<(unsigned)T, (unsigned)((H / 8 + 31) / 32 * 32), 0, st>>>(
+        x, H, topk, w.row_of, w.xq, w.sxr, w.out, dbg ? dbg->qx : nullptr, dbg ? dbg->sx : nullptr);
+    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+
+    const int max_active = (int)(R < E ? R : E);
+    const bool wide = R > (int64_t)E * 8;   // more than 8 rows per expert on average
+    MoeGemmArgs g1 = {};
+    g1.w = w13;
+    g1.sw = s13;
+    g1.xq = w.xq;
+    g1.sxr = w.sxr;
+    g1.counts = w.counts;
+    g1.offsets = w.offsets;
+    g1.active = w.active;
+    g1.n_active = w.n_active;
+    g1.rows = 2 * I;
+    g1.K = H;
+    g1.a_out = w.a;
+    rc = wide ? launch_moe_gemm<2, 4, 4, true>(g1, (2 * I) / 32, max_active, st)
+              : launch_moe_gemm<2, 4, 1, true>(g1, (2 * I) / 32, max_active, st);
+    if (rc != W8A8_OK) return rc;
+
+    cudaError_t e = launch_quant_rows<float>(w.a, R, I, I, w.qa, I, w.sa, st, current_sms());
+    if (e != cudaSuccess) return W8A8_ERR_CUDA;
+
+    MoeGemmArgs g2 = {};
+    g2.w = w2;
+    g2.sw = s2;
+    g2.xq = w.qa;
+    g2.sxr = w.sa;
+    g2.counts = w.counts;
+    g2.offsets = w.offsets;
+    g2.active = w.active;
+    g2.n_active = w.n_active;
+    g2.rows = H;
+    g2.K = I;
+    g2.row_tok = w.row_tok;
+    g2.row_w = w.row_w;
+    g2.out_f32 = w.out;
+    rc = wide ? launch_moe_gemm<8, 1, 4, false>(g2, H / 128, max_active, st)
+              : launch_moe_gemm<8, 1, 1, false>(g2, H / 128, max_active, st);
+    if (rc != W8A8_OK) return rc;
+
+    const int64_t n = T * H;
+    moe_finalize_kernel<<<(unsigned)((n / 4 + 255) / 256 + 1), 256, 0, st>>>(w.out, y, n);
+    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+
+    if (dbg) {
+        if (dbg->topk_ids && cudaMemcpyAsync(dbg->topk_ids, w.ids, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->topk_w && cudaMemcpyAsync(dbg->topk_w, w.wts, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->counts && cudaMemcpyAsync(dbg->counts, w.counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->qa || dbg->sa) {
+            moe_debug_gather_kernel<<<(unsigned)R, 128, 0, st>>>(w.qa, w.sa, w.row_of, R, I, dbg->qa, dbg->sa);
+            if ((rc = last_launch_status()) != W8A8_OK) return rc;
+        }
+    }
+    return W8A8_OK;
+}
+
+// ----------------------------------------------------------------- FWHT128
+int fwht128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, void* stream) {
+    if (!x || !q || !s || M <= 0 || K <= 0 || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 2)) return W8A8_ERR_INVALID_ARG;
+    const int64_t blocks = M * (K / 128);
+    const int64_t ctas = (blocks + 7) / 8;
+    if (ctas > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
+    fwht128_quant_kernel<<<(unsigned)ctas, 256, 0, (cudaStream_t)stream>>>(x, M, K, q, s);
+    return last_launch_status();
+}
+
+int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
+                     int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!qx || !sx || !qw || !sw || !y) return W8A8_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(M, N, K) || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sx, 2) || !aligned(sw, 2))
+        return W8A8_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (M <= 8) {
+        if (K / 128 > kG128MaxGroups || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
+        gemv_g128_kernel<<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K);
+        return last_launch_status();
+    }
+    TcParams p = {};
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.gsx = sx;
+    p.gsw = sw;
+    p.out = y;
+    return launch_tc<128, 6, kEpiG128, 4>(qx, qw, p, st);
+}
+
+// ----------------------------------------------------------------- diagnostics
+int w8a8_exp_proj(const float* x, float* y, int64_t n, void* stream) {
+    if (!x || !y || n <= 0) return W8A8_ERR_INVALID_ARG;
+    exp_proj_kernel<<<(unsigned)((n + 255) / 256), 256, 0, (cudaStream_t)stream>>>(x, y, n);
+    return last_launch_status();
+}
+
+int w8a8_get_device_error(void* stream, int* site) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return W8A8_ERR_CUDA;
+    int err = 0, where = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&err, g_device_error, sizeof(int)) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&where, g_device_error_site, sizeof(int)) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_device_error_site, &zero, sizeof(int)) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (site) *site = where;
+    return err;
+}
+
+int w8a8_debug_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000LL) return W8A8_ERR_INVALID_ARG;
+    debug_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_ns);
+    return last_launch_status();
+}
+
+}  // extern "C"

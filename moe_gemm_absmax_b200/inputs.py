@@ -95,3 +95,18 @@ def hadamard_linear(seed: int, M: int, K: int = 2048, N: int = 4096,
     x = activations(rng, M, K, n_outlier, factor)
     w = weights(rng, (N, K))
     return to_bf16_bits(x), to_bf16_bits(w)
+
+
+def moe_weights(seed: int, E: int = 256, H: int = 2048, I: int = 512):
+    """Expert weights drawn from their own stream, so that one set serves every
+    token count: w13 fp32 [E,2I,H] (row 2i gate_i, row 2i+1 up_i), w2 fp32 [E,H,I]."""
+    rng = np.random.default_rng([seed, 1])
+    return weights(rng, (E, 2 * I, H)), weights(rng, (E, H, I))
+
+
+def moe_tokens(seed: int, T: int, E: int = 256, H: int = 2048):
+    """x ~ N(0,1) bf16 [T,H] and router logits ~ N(0,1) bf16 [T,E]."""
+    rng = np.random.default_rng([seed, 2, T])
+    x = rng.standard_normal((T, H), dtype=np.float32)
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    return to_bf16_bits(x), to_bf16_bits(logits)

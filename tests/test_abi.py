@@ -1,0 +1,65 @@
+"""The C-ABI library loads and exports every entry point the header
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_gemm_absmax_b200 import build, w8a8
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "w8a8.h")).read()
+    return sorted(set(re.findall(r"^W8A8_API\s+[\w\s\*]+?\b((?:w8a8|fwht128)_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return w8a8.lib()
+
+
+def test_header_declares_the_four_named_entry_points():
+    names = _declared()
+    for n in ("w8a8_quant_act", "w8a8_linear", "w8a8_moe_forward", "fwht128_quant"):
+        assert n in names
+    assert set(names) == set(w8a8.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in _declared():
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    assert w8a8.status_str(0) == "ok"
+    assert w8a8.status_str(-2) == "workspace too small"
+    assert "sm_100a" in w8a8.version()
+
+
+def test_workspace_queries(L):
+    assert L.w8a8_linear_workspace_size(8, 5120, 17408) >= 8 * 17408 + 32
+    assert L.w8a8_linear_workspace_size(0, 5, 5) == 0
+    assert L.w8a8_moe_workspace_size(4096, 256, 2048, 512, 8) > 4096 * 8 * 2048
+    assert L.w8a8_gemm_workspace_size(4096, 5120, 17408, w8a8.PATH_TCGEN05) == 0
+
+
+def test_argument_checks_without_gpu(L):
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    # null pointers, bad sizes, misalignment: rejected before anything is enqueued
+    assert L.w8a8_quant_act(None, 4, 64, 64, fake, fake, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_quant_act(fake, 4, 60, 64, fake, fake, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_quant_act(vp(0x10001), 4, 64, 64, fake, fake, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_linear(fake, fake, fake, fake, 4, 12, 64, fake, 1 << 20, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_linear(fake, fake, fake, fake, 4, 16, 64, fake, 16, None) == w8a8.ERR_WORKSPACE
+    assert L.fwht128_quant(fake, 2, 192, fake, fake, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_moe_forward(fake, fake, fake, fake, fake, fake, fake, 4, 8, 256, 64, 9, fake, 1 << 30,
+                              None, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_moe_forward(fake, fake, fake, fake, fake, fake, fake, 4, 8, 256, 64, 2, fake, 64,
+                              None, None) == w8a8.ERR_WORKSPACE
+    assert L.w8a8_gemm_q(fake, fake, fake, fake, fake, 4, 16, 64, 7, None, 0, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_debug_wait_timeout(10, None) == w8a8.ERR_INVALID_ARG

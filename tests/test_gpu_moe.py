@@ -1,0 +1,99 @@
+"""GPU parity of the routed W8A8 MoE layer (a5 .. a11) against the CPU
+oracle: expert ids, histogram, x codes and the gated intermediate's codes
+and scales bit for bit; routing weights to fp32 rounding; the bf16 output
+within one bf16 ulp plus the reassociation bound of the fp32 combine."""
+import numpy as np
+import pytest
+import torch
+
+from moe_gemm_absmax_b200 import inputs, w8a8
+from tests._util import assert_bf16_close, from_dev_bf16, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _quant_experts_gpu(w13, w2):
+    q13, s13 = w8a8.quant_rows_f32(_dev(w13))
+    q2, s2 = w8a8.quant_rows_f32(_dev(w2))
+    return q13, s13, q2, s2
+
+
+def _quant_experts_orc(orc, w13, w2):
+    E, I2, H = w13.shape
+    q13, s13 = orc.quant_rows_f32(w13.reshape(E * I2, H))
+    q2, s2 = orc.quant_rows_f32(w2.reshape(E * H, -1))
+    return q13.reshape(w13.shape), s13.reshape(E, I2), q2.reshape(w2.shape), s2.reshape(E, H)
+
+
+def _compare(orc, xb, lb, gpu_w, orc_w, topk, tokens):
+    q13, s13, q2, s2 = gpu_w
+    y, dbg = w8a8.moe_forward(to_dev_bf16(xb), to_dev_bf16(lb), q13, s13, q2, s2, topk, debug=True)
+    y = from_dev_bf16(y)
+    ids_all, _ = orc.route(lb, topk)
+    E = q13.shape[0]
+    assert np.array_equal(dbg["counts"].cpu().numpy(), np.bincount(ids_all.reshape(-1), minlength=E))
+    assert np.array_equal(dbg["topk_ids"].cpu().numpy(), ids_all)
+    ref = orc.moe_forward(xb, lb, *orc_w, topk, tokens=tokens)
+    t = ref["tokens"]
+    assert np.array_equal(dbg["topk_ids"].cpu().numpy()[t], ref["ids"])
+    assert np.allclose(dbg["topk_w"].cpu().numpy()[t], ref["wts"], rtol=8 * 2.0 ** -24, atol=0)
+    assert np.array_equal(dbg["qx"].cpu().numpy()[t], ref["qx"])
+    assert np.array_equal(dbg["sx"].cpu().numpy()[t].view(np.uint32), ref["sx"].view(np.uint32))
+    assert np.array_equal(dbg["qa"].cpu().numpy()[t], ref["qa"])
+    assert np.array_equal(dbg["sa"].cpu().numpy()[t].view(np.uint32), ref["sa"].view(np.uint32))
+    # the k fp32 contributions may be added in any order
+    assert_bf16_close(y[t], ref["y32"], extra=2.0 ** -18 * ref["yabs"].astype(np.float64), what="moe y")
+
+
+def _small(seed, T, E, H, I, skew=None):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    if skew is not None:
+        logits[:, skew] += 6.0
+    w13 = inputs.weights(rng, (E, 2 * I, H))
+    w2 = inputs.weights(rng, (E, H, I))
+    return inputs.to_bf16_bits(x), inputs.to_bf16_bits(logits), w13, w2
+
+
+@pytest.mark.parametrize("T,E,H,I,k,skew", [(5, 8, 256, 64, 2, None), (37, 8, 256, 64, 2, None),
+                                             (40, 16, 512, 128, 2, 3), (1, 4, 128, 64, 4, None),
+                                             (9, 256, 2048, 512, 8, None)])
+def test_moe_small_configs(orc, T, E, H, I, k, skew):
+    xb, lb, w13, w2 = _small(T * 31 + E, T, E, H, I, skew)
+    gw = _quant_experts_gpu(w13, w2)
+    ow = _quant_experts_orc(orc, w13, w2)
+    assert np.array_equal(gw[0].cpu().numpy(), ow[0]) and np.array_equal(gw[2].cpu().numpy(), ow[2])
+    _compare(orc, xb, lb, gw, ow, k, None)
+
+
+def test_moe_zero_token_row(orc):
+    xb, lb, w13, w2 = _small(3, 6, 8, 256, 64)
+    xb[4] = 0
+    gw = _quant_experts_gpu(w13, w2)
+    y = from_dev_bf16(w8a8.moe_forward(to_dev_bf16(xb), to_dev_bf16(lb), *gw, 2))
+    assert not y[4].any()
+
+
+@pytest.fixture(scope="module")
+def full_experts(orc):
+    w13, w2 = inputs.moe_weights(0)
+    gw = _quant_experts_gpu(w13, w2)
+    ow = _quant_experts_orc(orc, w13, w2)
+    assert np.array_equal(gw[0].cpu().numpy(), ow[0]) and np.array_equal(gw[1].cpu().numpy(), ow[1])
+    assert np.array_equal(gw[2].cpu().numpy(), ow[2]) and np.array_equal(gw[3].cpu().numpy(), ow[3])
+    del w13, w2
+    return gw, ow
+
+
+@pytest.mark.parametrize("T", [1, 8, 512, 4096])
+def test_moe_full_size(orc, full_experts, T):
+    gw, ow = full_experts
+    xb, lb = inputs.moe_tokens(0, T)
+    rng = np.random.default_rng(T)
+    tokens = None if T <= 8 else np.unique(np.concatenate([rng.integers(0, T, 24), [0, T - 1]]))
+    _compare(orc, xb, lb, gw, ow, 8, tokens)
