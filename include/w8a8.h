@@ -89,6 +89,30 @@ W8A8_API size_t w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 W8A8_API int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* y, int64_t M, int64_t N, int64_t K,
                 void* ws, size_t ws_bytes, void* stream);
 
+/* Dense W8A8 linear for callers that cannot allocate device memory.
+ * No counterpart on the pages: an interface addition of this library.
+ * Some callers cannot call cudaMalloc where they run the layer (an allocator
+ * locked during a step, a plugin host that only passes its input and output
+ * buffers).  This entry point computes exactly what w8a8_linear computes, with
+ * the same kernels, but keeps the scratch (activation codes and scales, split-K
+ * partials and counters) in a file-scope device array of
+ * W8A8_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.  It allocates nothing.
+ *   - Sizes: w8a8_linear_noalloc_scratch_size(M, N, K) must not exceed
+ *     W8A8_NOALLOC_SCRATCH_BYTES (4 MiB: e.g. M <= 8 at K = 17408, or
+ *     M * K up to about 4 million); larger calls return W8A8_ERR_UNSUPPORTED
+ *     and enqueue nothing.
+ *   - The first call on a device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (what
+ *     must start at zero is cleared by each call): calls that overlap on the GPU
+ *     (different streams, or different host threads on one device) race and
+ *     must be serialized by the caller. */
+#define W8A8_NOALLOC_SCRATCH_BYTES (4u << 20)
+W8A8_API size_t w8a8_linear_noalloc_scratch_size(int64_t M, int64_t N, int64_t K);
+W8A8_API int w8a8_linear_noalloc(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* y, int64_t M,
+                                 int64_t N, int64_t K, void* stream);
+
 /* GEMM on pre-quantized activations with the dequant epilogue (a2 + a3):
  *   qx int8 [M, K], sx fp32 [M], qw int8 [N, K], sw fp32 [N] -> y bf16 [M, N].
  * `path` is one of W8A8_PATH_*.  The GEMV path with M > 8 and K split over

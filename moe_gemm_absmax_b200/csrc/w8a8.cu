@@ -368,6 +368,57 @@ int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* 
     return run_tc(qx, sx, qw, sw, y, M, N, K, kEpiBf16, st);
 }
 
+// ----------------------------------------------------------------- linear without caller workspace
+// Some callers cannot allocate device memory at the point where they run the
+// layer (an allocator that is locked while a step runs, a plugin host that
+// only hands over its input and output buffers, code that must not touch the
+// allocator's state).  For them w8a8_linear_noalloc keeps w8a8_linear's
+// scratch -- the activation codes and scales and the GEMV's split-K partials
+// and arrival counters -- in this file-scope device array instead of a
+// caller-provided workspace.  Every GPU that loads the library holds the array
+// until the process exits.
+static __device__ __align__(256) uint8_t g_linear_noalloc_scratch[W8A8_NOALLOC_SCRATCH_BYTES];
+
+}  // extern "C"
+
+namespace {
+// Device address of g_linear_noalloc_scratch, looked up once per device with
+// that device current (the host-side symbol is only a stand-in, never a
+// device address).
+uint8_t* noalloc_scratch_ptr(int dev) {
+    static uint8_t* ptrs[kMaxDevices] = {nullptr};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_linear_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        ptrs[dev] = reinterpret_cast<uint8_t*>(p);
+    }
+    return ptrs[dev];
+}
+}  // namespace
+
+extern "C" {
+
+size_t w8a8_linear_noalloc_scratch_size(int64_t M, int64_t N, int64_t K) {
+    return w8a8_linear_workspace_size(M, N, K);
+}
+
+int w8a8_linear_noalloc(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* y, int64_t M, int64_t N,
+                        int64_t K, void* stream) {
+    if (!x || !qw || !sw || !y) return W8A8_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(M, N, K)) return W8A8_ERR_INVALID_ARG;
+    if (w8a8_linear_workspace_size(M, N, K) > (size_t)W8A8_NOALLOC_SCRATCH_BYTES) return W8A8_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    uint8_t* scratch = noalloc_scratch_ptr(dev);
+    if (scratch == nullptr) return W8A8_ERR_CUDA;
+    // The same kernels as w8a8_linear, on the static scratch; the quant kernel
+    // clears the split-K counters each call, so earlier contents do not matter.
+    return w8a8_linear(x, qw, sw, y, M, N, K, scratch, (size_t)W8A8_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int path) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
     const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8 && N % 16 == 0);

@@ -22,6 +22,7 @@ PATH_AUTO, PATH_TCGEN05, PATH_GEMV = 0, 1, 2
 # Every function the header include/w8a8.h declares.
 EXPORTS = (
     "w8a8_quant_act", "w8a8_quant_rows_f32", "w8a8_linear_workspace_size", "w8a8_linear",
+    "w8a8_linear_noalloc_scratch_size", "w8a8_linear_noalloc",
     "w8a8_gemm_workspace_size", "w8a8_gemm_q", "w8a8_gemm_s32", "w8a8_moe_workspace_size",
     "w8a8_moe_forward", "fwht128_quant", "w8a8_linear_g128", "w8a8_exp_proj",
     "w8a8_get_device_error", "w8a8_debug_wait_timeout", "w8a8_status_str", "w8a8_version",
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         "w8a8_quant_rows_f32": ([vp, i64, i64, vp, vp, vp], i32),
         "w8a8_linear_workspace_size": ([i64, i64, i64], sz),
         "w8a8_linear": ([vp, vp, vp, vp, i64, i64, i64, vp, sz, vp], i32),
+        "w8a8_linear_noalloc_scratch_size": ([i64, i64, i64], sz),
+        "w8a8_linear_noalloc": ([vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "w8a8_gemm_workspace_size": ([i64, i64, i64, i32], sz),
         "w8a8_gemm_q": ([vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp], i32),
         "w8a8_gemm_s32": ([vp, vp, vp, i64, i64, i64, i32, vp, sz, vp], i32),
@@ -158,6 +161,29 @@ def linear(x: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, y: torch.Tensor 
         ws = _workspace(need, x.device)
     _check(lib().w8a8_linear(_ptr(x), _ptr(qw), _ptr(sw), _ptr(y), M, N, K, _ptr(ws), ws.numel(),
                              _stream(stream)), "w8a8_linear")
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def linear_noalloc(x: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, y: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """The dense W8A8 linear for callers that cannot allocate device memory
+    while it runs: same result as :func:`linear`, scratch kept in the
+    library's static device array (at most NOALLOC_SCRATCH_BYTES), so only
+    x, the weights and y are passed.  Calls that overlap on the GPU race on
+    that array; the first call on a device must come before stream capture.
+    (The output tensor is allocated here only when the caller passes none.)"""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(qw, torch.int8, "qw", 2)
+    _need(sw, torch.float32, "sw", 1)
+    M, K = x.shape
+    N = qw.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().w8a8_linear_noalloc(_ptr(x), _ptr(qw), _ptr(sw), _ptr(y), M, N, K, _stream(stream)),
+           "w8a8_linear_noalloc")
     return y
 
 
