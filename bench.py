@@ -105,12 +105,15 @@ class ClockSampler:
 # --------------------------------------------------------------------------- timing helpers
 def time_events(torch, fn, iters, flush=None):
     """Mean device time of fn() per call in ms, CUDA events on the current stream,
-    one event pair per call; optional L2 flush between calls (outside the events)."""
+    one event pair per call; optional L2 flush between calls (outside the events).
+    A short device-side sleep before the start event keeps the GPU busy while
+    the host enqueues fn(), so no launch gap is timed."""
     st = torch.cuda.current_stream()
     ts = []
     for _ in range(iters):
         if flush is not None:
             flush()
+        torch.cuda._sleep(200000)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(st)
@@ -122,10 +125,12 @@ def time_events(torch, fn, iters, flush=None):
 
 
 def make_flush(torch, dev):
-    buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    """Evicts L2 by reading a buffer twice its size (a read leaves no dirty
+    lines whose write-back would compete with the next timed kernel)."""
+    buf = torch.ones(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     def flush():
-        buf.fill_(1)
+        buf.max()
     return flush
 
 

@@ -58,9 +58,9 @@ extern "C" {
 #define W8A8_ERR_TIMEOUT (-5)      /* a device-side bounded wait gave up */
 
 /* Selects the GEMM kernel in w8a8_gemm_q / w8a8_gemm_s32. */
-#define W8A8_PATH_AUTO 0      /* GEMV for M <= 8 and N % 16 == 0, tensor-core GEMM otherwise */
-#define W8A8_PATH_TCGEN05 1   /* tcgen05 kind::i8 GEMM, any M */
-#define W8A8_PATH_GEMV 2      /* weight-streaming GEMV, M <= 32, N % 16 == 0 */
+#define W8A8_PATH_AUTO 0      /* decode GEMV for M <= 8, tiled tensor-core GEMM otherwise */
+#define W8A8_PATH_TCGEN05 1   /* tiled tcgen05 kind::i8 GEMM (128-token tiles), any M */
+#define W8A8_PATH_GEMV 2      /* weight-streaming swap-AB tcgen05 GEMV, M <= 32 */
 
 /* ---------------------------------------------------------------------------
  * Per-token dynamic activation quantization (a1) -- [ATOM] "Precision split",

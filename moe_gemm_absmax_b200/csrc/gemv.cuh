@@ -61,7 +61,7 @@ struct GemvShape {
 // the final sums for their row block (warps with wk == 0 of the finishing CTA).
 // kseg / nkseg: this CTA's share of a K range split over nkseg CTAs;
 // ctr: this CTA's arrival counter slot (nkseg > 1).
-template <int WN, int WK, int TG, class RowMap>
+template <int WN, int WK, int TG, class RowMap, int U = kGemvUnroll, bool PF = false>
 __device__ __forceinline__ bool gemv_core(const GemvShape& a, int (&acc)[TG][4], int& block_out, int kseg = 0,
                                           int nkseg = 1, int ctr = 0) {
     static_assert(WN * WK == kGemvThreads / 32, "8 warps");
@@ -88,21 +88,37 @@ __device__ __forceinline__ bool gemv_core(const GemvShape& a, int (&acc)[TG][4],
     if (block_ok) {
         const int8_t* wr0 = a.w + RowMap::row(block, g) * a.K + 16 * t;
         const int8_t* wr1 = a.w + RowMap::row(block, g + 8) * a.K + 16 * t;
-        for (int c = c0; c < c1; c += kGemvUnroll) {
-            uint4 wa[kGemvUnroll], wb[kGemvUnroll];
+        uint4 wa[U], wb[U];
+        auto load = [&](int c, uint4 (&xa)[U], uint4 (&xb)[U]) {
 #pragma unroll
-            for (int u = 0; u < kGemvUnroll; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int k = (c + u) * 64 + 16 * t;
                 if (c + u < c1 && k < a.K) {
-                    wa[u] = ld_stream_16(wr0 + (int64_t)(c + u) * 64);
-                    wb[u] = ld_stream_16(wr1 + (int64_t)(c + u) * 64);
+                    xa[u] = ld_stream_16(wr0 + (int64_t)(c + u) * 64);
+                    xb[u] = ld_stream_16(wr1 + (int64_t)(c + u) * 64);
                 } else {
-                    wa[u] = make_uint4(0, 0, 0, 0);
-                    wb[u] = make_uint4(0, 0, 0, 0);
+                    xa[u] = make_uint4(0, 0, 0, 0);
+                    xb[u] = make_uint4(0, 0, 0, 0);
                 }
             }
+        };
+        if (PF) load(c0, wa, wb);
+        bool waited = false;
+        for (int c = c0; c < c1; c += U) {
+            uint4 na[U], nb[U];
+            if (PF) {
+                // issue the next batch of weight loads before this batch's MMAs
+                if (c + U < c1) load(c + U, na, nb);
+            } else {
+                load(c, wa, wb);
+            }
+            if (!waited) {
+                // weights never depend on the previous kernel; the codes do
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                waited = true;
+            }
 #pragma unroll
-            for (int u = 0; u < kGemvUnroll; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int k = (c + u) * 64 + 16 * t;
 #pragma unroll
                 for (int tg = 0; tg < TG; ++tg) {
@@ -118,7 +134,17 @@ __device__ __forceinline__ bool gemv_core(const GemvShape& a, int (&acc)[TG][4],
                     mma_s8_16832(acc[tg], A2, B2);
                 }
             }
+            if (PF) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    wa[u] = na[u];
+                    wb[u] = nb[u];
+                }
+            }
         }
+        if (!waited) asm volatile("griddepcontrol.wait;" ::: "memory");
+    } else {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
     }
 
     if (WK > 1) {
@@ -192,11 +218,11 @@ struct GemvEpiDense {
     int s32;           // 1: raw int32
 };
 
-template <int WN, int WK, int TG>
+template <int WN, int WK, int TG, int U>
 __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(GemvShape a, GemvEpiDense e) {
     int acc[TG][4];
     int block;
-    if (!gemv_core<WN, WK, TG, RowMapDense>(a, acc, block, blockIdx.y, gridDim.y, blockIdx.x)) return;
+    if (!gemv_core<WN, WK, TG, RowMapDense, U>(a, acc, block, blockIdx.y, gridDim.y, blockIdx.x)) return;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int tg = 0; tg < TG; ++tg) {
@@ -216,4 +242,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(GemvShape a, G
     }
 }
 
+
 }  // namespace w8a8
+
+

@@ -61,6 +61,9 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
                                                         int8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
                                                         int vpc, int cl, int* zero_buf, int zero_n) {
     using VT = VecTraits<Tin>;
+    // let a kernel launched after this one with programmatic serialization
+    // start its independent prologue now (it still waits for our results)
+    asm volatile("griddepcontrol.launch_dependents;");
     // optional side job: clear a small int buffer that a later kernel on the
     // same stream expects to find zero (split-K arrival counters)
     for (int i = blockIdx.x * NT + threadIdx.x; i < zero_n; i += gridDim.x * NT) zero_buf[i] = 0;

@@ -13,6 +13,7 @@
 #include "fwht.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_tc.cuh"
 #include "moe.cuh"
 #include "quant.cuh"
 #include "w8a8.h"
@@ -129,88 +130,150 @@ int run_tc(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw,
 }
 
 // ----------------------------------------------------------------- GEMV
+// Decode GEMV.  M <= 8: the register-streaming mma.sync kernel
+// (gemv_dense_kernel): 4 row blocks x 2 K-halves per CTA, 8 chunks of
+// weight loads in flight per thread, and the K range split over `nkseg`
+// CTAs when the rows alone give too few CTAs (measured fastest for both
+// decode shapes).  9 <= M <= 32: the swap-AB tcgen05 kernel (gemv_tc_kernel),
+// whose token columns grow for free.  Plans are fixed per shape
+// (independent of the device) so that workspace sizes are too.
 struct GemvPlan {
-    int wn, wk, tg, nkseg;
-    int ctas_x;        // CTAs along the rows
+    bool tc;           // tcgen05 swap-AB kernel
+    // register kernel
+    int tg;            // token groups of 8
+    int ctas_x;        // CTAs along the rows (4 row blocks each)
+    int nkseg;         // CTAs along K
+    // tcgen05 kernel
+    int bn, grid, ngroups, nkb;
+    size_t part_bytes;
+    int counters;
 };
 
-// Fixed for a shape (independent of the device) so that workspace sizes are too.
+constexpr int kGemvWN = 4, kGemvWK = 2;
+constexpr int kGemvGrid = 148;
+constexpr int kGemvMaxM = 32;
+
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
-    GemvPlan g;
-    g.tg = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
-    g.wn = 1;
-    g.wk = 8;
-    const int64_t nchunks = (K + 63) / 64;
-    if (nchunks < 16) {          // short K: warps take separate row blocks
-        g.wn = 8;
-        g.wk = 1;
+    GemvPlan g = {};
+    g.tc = M > 8;
+    if (!g.tc) {
+        g.tg = 1;
+        const int64_t blocks = (N + 15) / 16;
+        g.ctas_x = (int)((blocks + kGemvWN - 1) / kGemvWN);
+        const int64_t nchunks = (K + 63) / 64;
+        int s = 1;
+        while (s < 8 && (int64_t)g.ctas_x * s < 160 && nchunks / (kGemvWK * s * 2) >= 8) s *= 2;
+        g.nkseg = s;
+        g.part_bytes = s > 1 ? align_up((size_t)s * blocks * g.tg * 32 * 16, 256) : 0;
+        g.counters = s > 1 ? g.ctas_x : 0;
+    } else {
+        g.bn = M <= 16 ? 16 : 32;
+        g.ngroups = (int)((N + kGcBM - 1) / kGcBM);
+        g.nkb = (int)((K + kGcBK - 1) / kGcBK);
+        const int64_t units = (int64_t)g.ngroups * g.nkb;
+        g.grid = (int)(units < kGemvGrid ? units : kGemvGrid);
+        g.part_bytes = align_up((size_t)g.grid * 2 * kGcBM * g.bn * 4, 256);
+        g.counters = g.ngroups * 4;
     }
-    const int64_t blocks = (N + 15) / 16;
-    g.ctas_x = (int)((blocks + g.wn - 1) / g.wn);
-    const int64_t target = 148 * 8;   // ~8 resident CTAs per SM over the 148 SMs of a B200
-    int s = 1;
-    while (s < 8 && (int64_t)g.ctas_x * s * 2 <= target + target / 2 && nchunks / (g.wk * s * 2) >= 2) s *= 2;
-    g.nkseg = s;
     return g;
 }
 
-size_t gemv_ws_bytes(const GemvPlan& g, int64_t N) {
-    if (g.nkseg == 1) return 0;
-    const int64_t blocks = (N + 15) / 16;
-    return align_up((size_t)g.nkseg * blocks * g.tg * 32 * 16, 256) + align_up((size_t)g.ctas_x * 4, 256);
+int gemv_counter_count(const GemvPlan& g) { return g.counters; }
+
+size_t gemv_ws_bytes(const GemvPlan& g) { return g.part_bytes + align_up((size_t)g.counters * 4, 256); }
+
+int* gemv_counters(const GemvPlan& g, void* scratch) {
+    return g.counters ? reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(scratch) + g.part_bytes) : nullptr;
 }
 
-template <int WN, int WK, int TG>
-int launch_gemv_t(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g, cudaStream_t st) {
-    dim3 grid((unsigned)g.ctas_x, (unsigned)g.nkseg, 1);
-    gemv_dense_kernel<WN, WK, TG><<<grid, kGemvThreads, 0, st>>>(a, e);
-    return last_launch_status();
+// Launch attribute: right after this library's activation-quant kernel (whose
+// inputs were complete before it started), the weight stream may begin while
+// that kernel finishes; codes, scales and counters are read only after it.
+// Otherwise plain stream order.
+void pdl_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* at, bool after_quant) {
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = after_quant ? 1 : 0;
 }
 
-int launch_gemv(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g, cudaStream_t st) {
-    if (g.wn == 1) {
-        if (g.tg == 1) return launch_gemv_t<1, 8, 1>(a, e, g, st);
-        if (g.tg == 2) return launch_gemv_t<1, 8, 2>(a, e, g, st);
-        return launch_gemv_t<1, 8, 4>(a, e, g, st);
+template <int BN>
+int launch_gemv_tc(const int8_t* qx, const int8_t* qw, const GemvTc& a, const GemvPlan& g, bool after_quant,
+                   cudaStream_t st) {
+    using SM = GcSmem<BN>;
+    auto kern = gemv_tc_kernel<BN>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    static bool attr_done[kMaxDevices] = {false};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        attr_done[dev] = true;
     }
-    if (g.tg == 1) return launch_gemv_t<8, 1, 1>(a, e, g, st);
-    if (g.tg == 2) return launch_gemv_t<8, 1, 2>(a, e, g, st);
-    return launch_gemv_t<8, 1, 4>(a, e, g, st);
+    CUtensorMap tw, tx;
+    if (!make_tmap_i8(&tw, qw, (uint64_t)a.N, (uint64_t)a.K, kGcBM)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tx, qx, (uint64_t)a.M, (uint64_t)a.K, BN)) return W8A8_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.grid, 1, 1);
+    cfg.blockDim = dim3(kGcThreads, 1, 1);
+    cfg.dynamicSmemBytes = SM::kBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    pdl_config(cfg, at, after_quant);
+    GemvTc args = a;
+    args.prefetch_w = after_quant ? 1 : 0;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tw, tx, args));
 }
 
-// Runs the GEMV given the split-K scratch (counters must be zero on entry).
+template <int TG, int U>
+int launch_gemv_reg(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g, bool after_quant, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.ctas_x, (unsigned)g.nkseg, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    pdl_config(cfg, at, after_quant);
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemv_dense_kernel<kGemvWN, kGemvWK, TG, U>, a, e));
+}
+
+// Runs the GEMV; `scratch` holds the partials and the counters (zero on entry).
 int run_gemv(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M, int64_t N,
-             int64_t K, bool s32, const GemvPlan& g, void* scratch, cudaStream_t st) {
-    GemvShape a;
-    a.w = qw;
-    a.x = qx;
-    a.tokens = (int)M;
-    a.rows = (int)N;
-    a.K = (int)K;
-    a.nchunks = (int)((K + 63) / 64);
-    a.part = nullptr;
-    a.counters = nullptr;
-    if (g.nkseg > 1) {
-        const int64_t blocks = (N + 15) / 16;
+             int64_t K, bool s32, const GemvPlan& g, void* scratch, bool after_quant, cudaStream_t st) {
+    if (!g.tc) {
+        GemvShape a;
+        a.w = qw;
+        a.x = qx;
+        a.tokens = (int)M;
+        a.rows = (int)N;
+        a.K = (int)K;
+        a.nchunks = (int)((K + 63) / 64);
         a.part = reinterpret_cast<int32_t*>(scratch);
-        a.counters = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(scratch) +
-                                            align_up((size_t)g.nkseg * blocks * g.tg * 32 * 16, 256));
+        a.counters = gemv_counters(g, scratch);
+        GemvEpiDense e;
+        e.sx = sx;
+        e.sw = sw;
+        e.out = out;
+        e.M = (int)M;
+        e.N = (int)N;
+        e.s32 = s32 ? 1 : 0;
+        return launch_gemv_reg<1, 8>(a, e, g, after_quant, st);
     }
-    GemvEpiDense e;
-    e.sx = sx;
-    e.sw = sw;
-    e.out = out;
-    e.M = (int)M;
-    e.N = (int)N;
-    e.s32 = s32 ? 1 : 0;
-    return launch_gemv(a, e, g, st);
-}
-
-int* gemv_counters(const GemvPlan& g, int64_t N, void* scratch) {
-    if (g.nkseg == 1) return nullptr;
-    const int64_t blocks = (N + 15) / 16;
-    return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(scratch) +
-                                  align_up((size_t)g.nkseg * blocks * g.tg * 32 * 16, 256));
+    GemvTc a;
+    a.sx = sx;
+    a.sw = sw;
+    a.out = out;
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.ngroups = g.ngroups;
+    a.nkb = g.nkb;
+    a.s32 = s32 ? 1 : 0;
+    a.part = reinterpret_cast<int*>(scratch);
+    a.counters = gemv_counters(g, scratch);
+    a.prefetch_w = 0;
+    if (g.bn == 16) return launch_gemv_tc<16>(qx, qw, a, g, after_quant, st);
+    return launch_gemv_tc<32>(qx, qw, a, g, after_quant, st);
 }
 
 bool gemm_shape_ok(int64_t M, int64_t N, int64_t K) {
@@ -343,7 +406,7 @@ int w8a8_quant_rows_f32(const float* w, int64_t N, int64_t K, int8_t* q, float* 
 size_t w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
     size_t b = align_up((size_t)M * K, 256) + align_up((size_t)M * 4, 256);
-    if (M <= 8 && N % 16 == 0) b += gemv_ws_bytes(gemv_plan(M, N, K), N);
+    if (M <= 8) b += gemv_ws_bytes(gemv_plan(M, N, K));
     return b;
 }
 
@@ -358,13 +421,14 @@ int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* 
     int8_t* qx = reinterpret_cast<int8_t*>(ws);
     float* sx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + align_up((size_t)M * K, 256));
     void* scratch = reinterpret_cast<uint8_t*>(sx) + align_up((size_t)M * 4, 256);
-    const bool gemv = M <= 8 && N % 16 == 0;
+    const bool gemv = M <= 8;
     GemvPlan g = gemv_plan(M, N, K);
-    int* ctr = gemv ? gemv_counters(g, N, scratch) : nullptr;
+    int* ctr = gemv ? gemv_counters(g, scratch) : nullptr;
     if (K / 8 > (int64_t)8 * 256 * kQuantMaxVec) return W8A8_ERR_UNSUPPORTED;
-    cudaError_t e = launch_quant_rows<uint16_t>(x, M, K, K, qx, K, sx, st, current_sms(), ctr, ctr ? g.ctas_x : 0);
+    cudaError_t e =
+        launch_quant_rows<uint16_t>(x, M, K, K, qx, K, sx, st, current_sms(), ctr, ctr ? gemv_counter_count(g) : 0);
     if (e != cudaSuccess) return W8A8_ERR_CUDA;
-    if (gemv) return run_gemv(qx, sx, qw, sw, y, M, N, K, false, g, scratch, st);
+    if (gemv) return run_gemv(qx, sx, qw, sw, y, M, N, K, false, g, scratch, true, st);
     return run_tc(qx, sx, qw, sw, y, M, N, K, kEpiBf16, st);
 }
 
@@ -421,9 +485,9 @@ int w8a8_linear_noalloc(const uint16_t* x, const int8_t* qw, const float* sw, ui
 
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int path) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
-    const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8 && N % 16 == 0);
+    const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8);
     if (!gemv) return 0;
-    return gemv_ws_bytes(gemv_plan(M, N, K), N);
+    return gemv_ws_bytes(gemv_plan(M, N, K));
 }
 
 static int gemm_common(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M,
@@ -434,18 +498,18 @@ static int gemm_common(const int8_t* qx, const float* sx, const int8_t* qw, cons
     if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(out, 16)) return W8A8_ERR_INVALID_ARG;
     if (!s32 && (!aligned(sx, 4) || !aligned(sw, 16))) return W8A8_ERR_INVALID_ARG;
     if (path < W8A8_PATH_AUTO || path > W8A8_PATH_GEMV) return W8A8_ERR_INVALID_ARG;
-    const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8 && N % 16 == 0);
+    const bool gemv = (path == W8A8_PATH_GEMV) || (path == W8A8_PATH_AUTO && M <= 8);
     if (gemv) {
-        if (M > 32 || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
+        if (M > kGemvMaxM) return W8A8_ERR_UNSUPPORTED;
         GemvPlan g = gemv_plan(M, N, K);
-        const size_t need = gemv_ws_bytes(g, N);
-        if (need > 0) {
+        const size_t need = gemv_ws_bytes(g);
+        if (g.counters > 0) {
             if (!ws || !aligned(ws, 256)) return W8A8_ERR_INVALID_ARG;
             if (ws_bytes < need) return W8A8_ERR_WORKSPACE;
-            if (cudaMemsetAsync(gemv_counters(g, N, ws), 0, (size_t)g.ctas_x * 4, st) != cudaSuccess)
+            if (cudaMemsetAsync(gemv_counters(g, ws), 0, (size_t)gemv_counter_count(g) * 4, st) != cudaSuccess)
                 return W8A8_ERR_CUDA;
         }
-        return run_gemv(qx, sx, qw, sw, out, M, N, K, s32, g, ws, st);
+        return run_gemv(qx, sx, qw, sw, out, M, N, K, s32, g, ws, false, st);
     }
     return run_tc(qx, sx, qw, sw, out, M, N, K, s32 ? kEpiS32 : kEpiBf16, st);
 }

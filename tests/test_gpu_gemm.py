@@ -17,7 +17,8 @@ def _rand_codes(rng, r, c):
 
 
 @pytest.mark.parametrize("path", [w8a8.PATH_TCGEN05, w8a8.PATH_GEMV])
-@pytest.mark.parametrize("M,N,K", [(1, 16, 16), (3, 48, 96), (8, 512, 528), (13, 272, 1040), (32, 512, 5120)])
+@pytest.mark.parametrize("M,N,K", [(1, 16, 16), (3, 48, 96), (8, 512, 528), (13, 272, 1040), (32, 512, 5120),
+                                   (3, 40, 96), (17, 136, 2064), (8, 1152, 17408)])
 def test_gemm_s32_small(orc, path, M, N, K):
     rng = np.random.default_rng(M * 7 + N + K)
     a, b = _rand_codes(rng, M, K), _rand_codes(rng, N, K)
@@ -102,14 +103,13 @@ def test_linear_prefill_ragged_rows(orc):
     assert assert_bf16_close(from_dev_bf16(y), y32, what="ragged") == 1.0
 
 
-def test_gemv_rejects_rows_not_multiple_of_16():
-    a = torch.zeros(3, 96, dtype=torch.int8, device="cuda")
+def test_gemv_rejects_more_than_32_tokens():
+    a = torch.zeros(33, 96, dtype=torch.int8, device="cuda")
     b = torch.zeros(40, 96, dtype=torch.int8, device="cuda")
     with pytest.raises(w8a8.W8A8Error) as e:
         w8a8.gemm_s32(a, b, w8a8.PATH_GEMV)
     assert e.value.status == w8a8.ERR_UNSUPPORTED
-    # the automatic choice takes the tensor-core path for such N
-    assert w8a8.gemm_s32(a, b).shape == (3, 40)
+    assert w8a8.gemm_s32(a, b).shape == (33, 40)
 
 
 def test_linear_repeated_calls_and_workspace_reuse(orc):
