@@ -239,6 +239,13 @@ __device__ __forceinline__ int quant_code(float v, float s) {
     return max(-127, min(127, q));
 }
 
+// Four fp32 atomic adds in one vector reduction (16-byte aligned address).
+__device__ __forceinline__ void red_add_v4(float* addr, const float (&v)[4]) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+                 "f"(v[3])
+                 : "memory");
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
 __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {

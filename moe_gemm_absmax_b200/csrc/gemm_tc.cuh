@@ -33,17 +33,66 @@ constexpr int kTcBK = 128;          // int8 elements (= bytes) of K per stage: o
 constexpr int kTcThreads = 192;
 constexpr int kKernelIdGemmTc = 1;
 
-enum TcEpilogue : int { kEpiBf16 = 0, kEpiS32 = 1, kEpiG128 = 2 };
+// Epilogues: dense bf16, raw int32, group-128 promotion, and the two grouped
+// MoE epilogues (gated SiLU over interleaved gate/up columns; weighted
+// combine into the token's fp32 output row).
+enum TcEpilogue : int { kEpiBf16 = 0, kEpiS32 = 1, kEpiG128 = 2, kEpiMoeGated = 3, kEpiMoeCombine = 4 };
 
 struct TcParams {
     int M, N, K;
     int num_m_tiles, num_n_tiles, num_k_blocks;
-    const float* sx;        // [M]        (kEpiBf16)
-    const float* sw;        // [N]        (kEpiBf16)
+    const float* sx;        // [M]        (kEpiBf16; grouped: scale of each sorted row)
+    const float* sw;        // [N]        (kEpiBf16; grouped: [E, N] per-expert channel scales)
     const uint16_t* gsx;    // [M, G] bf16 (kEpiG128)
     const uint16_t* gsw;    // [N, G] bf16 (kEpiG128)
     void* out;              // bf16 or int32 [M, N], row stride N
+    // ---- grouped (MoE) mode: A = expert-sorted rows, B = per-expert weights [E * N, K]
+    const int32_t* counts;  // [E] rows of each expert
+    const int32_t* offsets; // [E + 1] first sorted row of each expert
+    const int32_t* tile_off;// [E + 1] prefix sum of ceil(counts / 128)
+    int E;
+    float* a_out;           // kEpiMoeGated: fp32 [M, N / 2]
+    const int32_t* row_tok; // kEpiMoeCombine: token of each sorted row
+    const float* row_w;     // kEpiMoeCombine: routing weight of each sorted row
+    float* out_f32;         // kEpiMoeCombine: fp32 [T, N]
 };
+
+// Coordinates of one output tile.
+struct TcTile {
+    int a_row;      // first A row (TMA y coordinate)
+    int b_row;      // first B row
+    int valid;      // rows of the tile that belong to it (<= 128)
+    int n0;         // first output column within the expert (or the matrix)
+    int e;          // expert (grouped) / 0
+};
+
+template <bool GROUPED, int BN>
+__device__ __forceinline__ TcTile tc_tile(const TcParams& p, int tile) {
+    TcTile t;
+    if (!GROUPED) {
+        const int mt = tile % p.num_m_tiles, nt = tile / p.num_m_tiles;
+        t.a_row = mt * kTcBM;
+        t.b_row = nt * BN;
+        t.valid = min(kTcBM, p.M - t.a_row);
+        t.n0 = nt * BN;
+        t.e = 0;
+    } else {
+        const int gm = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
+        int lo = 0, hi = p.E - 1;          // expert e with tile_off[e] <= gm < tile_off[e + 1]
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(p.tile_off + mid) <= gm) lo = mid;
+            else hi = mid - 1;
+        }
+        const int lm = gm - __ldg(p.tile_off + lo);
+        t.e = lo;
+        t.a_row = __ldg(p.offsets + lo) + lm * kTcBM;
+        t.valid = min(kTcBM, __ldg(p.counts + lo) - lm * kTcBM);
+        t.n0 = nt * BN;
+        t.b_row = lo * p.N + nt * BN;
+    }
+    return t;
+}
 
 template <int BN, int STAGES>
 struct TcSmem {
@@ -54,7 +103,7 @@ struct TcSmem {
     static constexpr int kBytes = 1024 /*alignment slack*/ + kTiles + kBars + 16;
 };
 
-template <int BN, int STAGES, int EPI, int NACC>
+template <int BN, int STAGES, int EPI, int NACC, bool GROUPED = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
@@ -105,7 +154,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+    const int num_tiles =
+        GROUPED ? __ldg(p.tile_off + p.E) * p.num_n_tiles : p.num_m_tiles * p.num_n_tiles;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -116,16 +166,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t last_phase = 0;      // bit s: phase of the last load into stage s
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                const int mt = tile % p.num_m_tiles;
-                const int nt = tile / p.num_m_tiles;
+                const TcTile ti = tc_tile<GROUPED, BN>(p, tile);
                 for (int kb = 0; kb < p.num_k_blocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, (kKernelIdGemmTc << 16) | 1)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(&full[stage], (uint32_t)(SM::kA + SM::kB));
-                    tma_load_2d(sA + stage * SM::kA, &tmA, &full[stage], kb * kTcBK, mt * kTcBM);
-                    tma_load_2d(sB + stage * SM::kB, &tmB, &full[stage], kb * kTcBK, nt * BN);
+                    tma_load_2d(sA + stage * SM::kA, &tmA, &full[stage], kb * kTcBK, ti.a_row);
+                    tma_load_2d(sB + stage * SM::kB, &tmB, &full[stage], kb * kTcBK, ti.b_row);
                     issued |= 1u << stage;
                     last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -203,10 +252,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-            const int mt = tile % p.num_m_tiles;
-            const int nt = tile / p.num_m_tiles;
-            const int row = mt * kTcBM + row_in_tile;
-            const bool row_ok = row < p.M;
+            const TcTile ti = tc_tile<GROUPED, BN>(p, tile);
+            const int nt = ti.n0 / BN;
+            const int row = ti.a_row + row_in_tile;
+            const bool row_ok = row_in_tile < ti.valid;
             const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
             if constexpr (EPI == kEpiG128) {
                 const int G = p.num_k_blocks;
@@ -261,7 +310,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) break;
                 tc_fence_after();
                 float sxr = 0.0f;
-                if (EPI == kEpiBf16 && row_ok) sxr = __ldg(p.sx + row);
+                if ((EPI == kEpiBf16 || EPI == kEpiMoeGated || EPI == kEpiMoeCombine) && row_ok) sxr = __ldg(p.sx + row);
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 32) {
                     uint32_t r[32];
@@ -269,6 +318,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_wait_ld();
                     const int n0 = nt * BN + c;
                     if (!row_ok || n0 >= p.N) continue;
+                    if (EPI == kEpiMoeGated) {
+                        // columns n0 .. n0+31 of expert e: 16 (gate, up) pairs
+                        const float* swe = p.sw + (int64_t)ti.e * p.N + n0;
+                        float* arow = p.a_out + (int64_t)row * (p.N / 2) + n0 / 2;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float av[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int j = 8 * q + 2 * i;
+                                const float vg = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), __ldg(swe + j));
+                                const float vu =
+                                    __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sxr), __ldg(swe + j + 1));
+                                av[i] = __fmul_rn(silu_proj(vg), vu);
+                            }
+                            *reinterpret_cast<float4*>(arow + 4 * q) = make_float4(av[0], av[1], av[2], av[3]);
+                        }
+                        continue;
+                    }
+                    if (EPI == kEpiMoeCombine) {
+                        const float* swe = p.sw + (int64_t)ti.e * p.N + n0;
+                        float* orow = p.out_f32 + (int64_t)__ldg(p.row_tok + row) * p.N + n0;
+                        const float wr = __ldg(p.row_w + row);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float cv[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int j = 4 * q + i;
+                                const float y2 = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), __ldg(swe + j));
+                                cv[i] = __fmul_rn(wr, y2);
+                            }
+                            red_add_v4(orow + 4 * q, cv);
+                        }
+                        continue;
+                    }
                     if (EPI == kEpiBf16) {
                         uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
                         const float4* swv = reinterpret_cast<const float4*>(p.sw + n0);

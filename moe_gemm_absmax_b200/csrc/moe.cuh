@@ -115,6 +115,7 @@ struct MoePlan {
     int32_t* offsets;    // [E + 1]
     int32_t* active;     // [E] touched experts, ascending
     int32_t* n_active;   // [1]
+    int32_t* tile_off;   // [E + 1] prefix sum of ceil(counts / 128): grouped-GEMM row tiles
     int32_t* row_of;     // [T * topk] expert-sorted row of (token, slot)
     int32_t* row_tok;    // [R] token of each sorted row
     int32_t* row_slot;   // [R] slot of each sorted row
@@ -183,6 +184,33 @@ __global__ void __launch_bounds__(1024) moe_plan_kernel(const int32_t* __restric
     }
     __syncthreads();
     if (e < E && c > 0) p.active[warp_tot[warp] + __popc(ball & ((1u << lane) - 1u))] = e;
+    // exclusive scan of the 128-row tiles of each expert
+    const int mt = (c + 127) / 128;
+    int tincl = mt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, tincl, o);
+        if (lane >= o) tincl += v;
+    }
+    __syncthreads();
+    if (lane == 31) warp_tot[warp] = tincl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += v;
+        }
+        warp_tot[lane] = wi - w;
+    }
+    __syncthreads();
+    if (e < E) {
+        const int texcl = tincl - mt + warp_tot[warp];
+        p.tile_off[e] = texcl;
+        if (e == E - 1) p.tile_off[E] = texcl + mt;
+    }
     // final rows and the per-row metadata of the sorted order
     for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
         const int r = off[ids[i]] + p.row_of[i];

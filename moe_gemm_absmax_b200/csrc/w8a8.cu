@@ -312,6 +312,7 @@ struct MoeWs {
     int32_t* offsets;
     int32_t* active;
     int32_t* n_active;
+    int32_t* tile_off;
     int32_t* row_of;
     int32_t* row_tok;
     int32_t* row_slot;
@@ -341,6 +342,7 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
     w.active = reinterpret_cast<int32_t*>(take((size_t)E * 4));
     w.n_active = reinterpret_cast<int32_t*>(take(4));
+    w.tile_off = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
     w.row_of = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.row_tok = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.row_slot = reinterpret_cast<int32_t*>(take((size_t)R * 4));
@@ -353,6 +355,33 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     w.out = reinterpret_cast<float*>(take((size_t)T * H * 4));
     w.bytes = o;
     return w;
+}
+
+// Grouped tcgen05 GEMM over the expert-sorted rows: A = sorted codes
+// [R, K], B = the experts' weights viewed as [E * N, K].
+template <int EPI>
+int launch_tc_grouped(const int8_t* A, int64_t rowsA, const int8_t* B, int E, TcParams p, cudaStream_t st) {
+    constexpr int BN = 256, STAGES = 4;
+    using SM = TcSmem<BN, STAGES>;
+    auto kern = gemm_i8_tc_kernel<BN, STAGES, EPI, 2, true>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    static bool attr_done[kMaxDevices] = {false};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    CUtensorMap ta, tb;
+    if (!make_tmap_i8(&ta, A, (uint64_t)rowsA, (uint64_t)p.K, kTcBM)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tb, B, (uint64_t)E * p.N, (uint64_t)p.K, BN)) return W8A8_ERR_CUDA;
+    p.E = E;
+    p.num_m_tiles = 0;
+    p.num_n_tiles = (p.N + BN - 1) / BN;
+    p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
+    kern<<<device_sms(dev), kTcThreads, SM::kBytes, st>>>(ta, tb, p);
+    return last_launch_status();
 }
 
 template <int WN, int WK, int TG, bool GATED>
@@ -550,7 +579,7 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     moe_route_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
-    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.row_of, w.row_tok, w.row_slot, w.row_w};
+    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.row_of, w.row_tok, w.row_slot, w.row_w};
     moe_plan_kernel<<<1, 1024, 0, st>>>(w.ids, w.wts, R, E, topk, plan);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
@@ -560,6 +589,36 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
 
     const int max_active = (int)(R < E ? R : E);
     const bool wide = R > (int64_t)E * 8;   // more than 8 rows per expert on average
+    // many rows per expert: grouped tcgen05 GEMMs over 128-row tiles of each expert's rows
+    const bool tiled = R >= (int64_t)E * 16 && (2 * I) % 256 == 0 && H % 256 == 0;
+    if (tiled) {
+        TcParams p1 = {};
+        p1.N = 2 * I;
+        p1.K = H;
+        p1.M = (int)R;
+        p1.sx = w.sxr;
+        p1.sw = s13;
+        p1.counts = w.counts;
+        p1.offsets = w.offsets;
+        p1.tile_off = w.tile_off;
+        p1.a_out = w.a;
+        if ((rc = launch_tc_grouped<kEpiMoeGated>(w.xq, R, w13, E, p1, st)) != W8A8_OK) return rc;
+        cudaError_t e2 = launch_quant_rows<float>(w.a, R, I, I, w.qa, I, w.sa, st, current_sms());
+        if (e2 != cudaSuccess) return W8A8_ERR_CUDA;
+        TcParams p2 = {};
+        p2.N = H;
+        p2.K = I;
+        p2.M = (int)R;
+        p2.sx = w.sa;
+        p2.sw = s2;
+        p2.counts = w.counts;
+        p2.offsets = w.offsets;
+        p2.tile_off = w.tile_off;
+        p2.row_tok = w.row_tok;
+        p2.row_w = w.row_w;
+        p2.out_f32 = w.out;
+        if ((rc = launch_tc_grouped<kEpiMoeCombine>(w.qa, R, w2, E, p2, st)) != W8A8_OK) return rc;
+    }
     MoeGemmArgs g1 = {};
     g1.w = w13;
     g1.sw = s13;
@@ -572,6 +631,7 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     g1.rows = 2 * I;
     g1.K = H;
     g1.a_out = w.a;
+    if (!tiled) {
     rc = wide ? launch_moe_gemm<2, 4, 4, true>(g1, (2 * I) / 32, max_active, st)
               : launch_moe_gemm<2, 4, 1, true>(g1, (2 * I) / 32, max_active, st);
     if (rc != W8A8_OK) return rc;
@@ -596,6 +656,7 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     rc = wide ? launch_moe_gemm<8, 1, 4, false>(g2, H / 128, max_active, st)
               : launch_moe_gemm<8, 1, 1, false>(g2, H / 128, max_active, st);
     if (rc != W8A8_OK) return rc;
+    }
 
     const int64_t n = T * H;
     moe_finalize_kernel<<<(unsigned)((n / 4 + 255) / 256 + 1), 256, 0, st>>>(w.out, y, n);
