@@ -140,8 +140,8 @@ W8A8_API int w8a8_gemm_s32(const int8_t* qx, const int8_t* qw, int32_t* acc, int
  * renormalised over the k; x quantized once per token (shared by its
  * experts); v = (float(qx . w13[e,r]) * sx) * s13[e,r];
  * a_i = SiLU(v_2i) * v_2i+1; (qa, sa) = per-row quant of a; y2_n =
- * (float(qa . w2[e,n]) * sa) * s2[e,n]; y = bf16( sum_j w_j * y2 ).  The
- * combine sums the k contributions in fp32 in an unspecified order.
+ * (float(qa . w2[e,n]) * sa) * s2[e,n]; y = bf16( sum_j w_j * y2 ) with the k
+ * contributions added in fp32 in slot order.
  * ws_bytes >= w8a8_moe_workspace_size(T, E, H, I, topk).  `dbg` may be NULL;
  * otherwise its non-NULL members receive intermediate values. */
 typedef struct w8a8_moe_debug {

@@ -240,9 +240,8 @@ __device__ __forceinline__ int quant_code(float v, float s) {
 }
 
 // Four fp32 atomic adds in one vector reduction (16-byte aligned address).
-__device__ __forceinline__ void red_add_v4(float* addr, const float (&v)[4]) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v[0]), "f"(v[1]), "f"(v[2]),
-                 "f"(v[3])
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
 

@@ -34,9 +34,16 @@ constexpr int kTcThreads = 192;
 constexpr int kKernelIdGemmTc = 1;
 
 // Epilogues: dense bf16, raw int32, group-128 promotion, and the two grouped
-// MoE epilogues (gated SiLU over interleaved gate/up columns; weighted
-// combine into the token's fp32 output row).
-enum TcEpilogue : int { kEpiBf16 = 0, kEpiS32 = 1, kEpiG128 = 2, kEpiMoeGated = 3, kEpiMoeCombine = 4 };
+// MoE epilogues (gated SiLU over interleaved gate/up columns; the routing-
+// weighted output of each sorted row, stored at its (token, slot)).
+enum TcEpilogue : int {
+    kEpiBf16 = 0,
+    kEpiS32 = 1,
+    kEpiG128 = 2,
+    kEpiMoeGated = 3,
+    kEpiMoeCombine = 4,        // w * y2 stored at (token, slot)
+    kEpiMoeCombineAtomic = 5   // w * y2 added atomically into the token's row
+};
 
 struct TcParams {
     int M, N, K;
@@ -53,8 +60,11 @@ struct TcParams {
     int E;
     float* a_out;           // kEpiMoeGated: fp32 [M, N / 2]
     const int32_t* row_tok; // kEpiMoeCombine: token of each sorted row
+    const int32_t* row_slot;// kEpiMoeCombine: slot of each sorted row
     const float* row_w;     // kEpiMoeCombine: routing weight of each sorted row
-    float* out_f32;         // kEpiMoeCombine: fp32 [T, N]
+    float* contrib;         // kEpiMoeCombine: fp32 [T * topk, N], row (token * topk + slot);
+                            // kEpiMoeCombineAtomic: fp32 [T, N]
+    int topk;
 };
 
 // Coordinates of one output tile.
@@ -103,9 +113,16 @@ struct TcSmem {
     static constexpr int kBytes = 1024 /*alignment slack*/ + kTiles + kBars + 16;
 };
 
-template <int BN, int STAGES, int EPI, int NACC, bool GROUPED = false>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// NEPI epilogue warps: 4 (one per TMEM lane quarter) or 8 (two per quarter,
+// each taking every other 32-column chunk) for epilogue-heavy tiles.
+template <int NEPI>
+constexpr int tc_threads() { return 64 + 32 * NEPI; }
+
+template <int BN, int STAGES, int EPI, int NACC, bool GROUPED = false, int NEPI = 4>
+__global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
     gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
+    static_assert(NEPI == 4 || NEPI == 8, "epilogue warps");
+    static_assert(NEPI == 4 || EPI != kEpiG128, "group-128 epilogue uses 4 warps");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(NACC >= 2 && NACC <= 4, "NACC");
     constexpr int kCols = NACC * BN;
@@ -136,7 +153,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], 32 * NEPI);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -247,6 +264,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;                 // TMEM lanes [32 q, 32 q + 32)
+        const int chalf = (warp - 2) / 4;             // NEPI == 8: which alternate 32-column chunks
         const int row_in_tile = quarter * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -310,9 +328,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) break;
                 tc_fence_after();
                 float sxr = 0.0f;
-                if ((EPI == kEpiBf16 || EPI == kEpiMoeGated || EPI == kEpiMoeCombine) && row_ok) sxr = __ldg(p.sx + row);
+                if ((EPI == kEpiBf16 || EPI == kEpiMoeGated || EPI == kEpiMoeCombine || EPI == kEpiMoeCombineAtomic) &&
+                    row_ok)
+                    sxr = __ldg(p.sx + row);
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
+                for (int c = (NEPI == 8 ? 32 * chalf : 0); c < BN; c += (NEPI == 8 ? 64 : 32)) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tq + (uint32_t)(acc * BN + c), r);
                     tc_wait_ld();
@@ -337,9 +357,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                         continue;
                     }
-                    if (EPI == kEpiMoeCombine) {
+                    if (EPI == kEpiMoeCombine || EPI == kEpiMoeCombineAtomic) {
                         const float* swe = p.sw + (int64_t)ti.e * p.N + n0;
-                        float* orow = p.out_f32 + (int64_t)__ldg(p.row_tok + row) * p.N + n0;
+                        constexpr bool at_slot = EPI == kEpiMoeCombine;
+                        const int64_t orow_i = at_slot
+                                                   ? (int64_t)__ldg(p.row_tok + row) * p.topk + __ldg(p.row_slot + row)
+                                                   : (int64_t)__ldg(p.row_tok + row);
+                        float* orow = p.contrib + orow_i * p.N + n0;
                         const float wr = __ldg(p.row_w + row);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
@@ -350,7 +374,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                 const float y2 = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), __ldg(swe + j));
                                 cv[i] = __fmul_rn(wr, y2);
                             }
-                            red_add_v4(orow + 4 * q, cv);
+                            if constexpr (at_slot)
+                                __stcs(reinterpret_cast<float4*>(orow + 4 * q), make_float4(cv[0], cv[1], cv[2], cv[3]));
+                            else
+                                red_add_v4(orow + 4 * q, cv[0], cv[1], cv[2], cv[3]);
                         }
                         continue;
                     }

@@ -5,21 +5,23 @@
 // Precision split: the router gate stays bf16.
 //
 // Kernels, in launch order:
-//   moe_route_kernel        one warp per token: fp32 softmax of the bf16
+//   moe_route_plan_kernel   one warp per token: fp32 softmax of the bf16
 //                           logits (project exp), top-k by logit with ties to
-//                           the lower expert index, weights renormalised
-//   moe_plan_kernel         one CTA: expert histogram, exclusive offsets,
-//                           list of touched experts, and the row of the
-//                           expert-sorted order each (token, slot) lands in
+//                           the lower expert index, weights renormalised, rank
+//                           of each (token, slot) inside its expert; the last
+//                           CTA scans the histogram (offsets, tile offsets,
+//                           touched experts)
 //   moe_quant_scatter_kernel  one CTA per token: per-token int8 quant of x,
 //                           codes written once per routed slot into the
-//                           expert-sorted code matrix; clears the fp32 output
+//                           expert-sorted code matrix; row metadata; clears
+//                           the token's fp32 output row
 //   gemm1 (grouped GEMV)    per touched expert: codes x w13^T, dequant,
 //                           SiLU(gate) * up -> fp32 intermediate
 //   requant                 per-row absmax int8 quant of the intermediate
-//   gemm2 (grouped GEMV)    codes x w2^T, dequant, times the routing weight,
-//                           fp32 atomic add into the token's output row
-//   moe_finalize_kernel     fp32 -> bf16
+//   gemm2 (grouped)         codes x w2^T, dequant, times the routing weight,
+//                           stored at (token, slot)
+//   moe_finalize_kernel     sum of each token's k contributions in slot order,
+//                           fp32, then bf16
 #pragma once
 
 #include <type_traits>
@@ -34,204 +36,177 @@ constexpr int kMoeMaxExperts = 1024;
 constexpr int kMoeMaxTopk = 32;
 
 // ---------------------------------------------------------------------------
-// a5: routing.  E <= 32 * EPL; lane l holds experts l, l + 32, ...
-template <int EPL>
-__global__ void __launch_bounds__(256) moe_route_kernel(const uint16_t* __restrict__ logits, int64_t T, int E,
-                                                        int topk, int32_t* __restrict__ ids,
-                                                        float* __restrict__ wts) {
-    const int lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= T) return;
-    float l[EPL], ex[EPL];
-    bool taken[EPL];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        l[i] = e < E ? bf16_bits_to_float(logits[t * E + e]) : -INFINITY;
-        if (isnan(l[i])) l[i] = -INFINITY;   // out of domain; keeps the selection well defined
-        taken[i] = e >= E;
-        mx = fmaxf(mx, l[i]);
-    }
-    mx = warp_max(mx);
-    float sum = 0.0f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        ex[i] = e < E ? exp_proj(__fsub_rn(l[i], mx)) : 0.0f;
-        sum = __fadd_rn(sum, ex[i]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
-
-    float psel_j = 0.0f;   // lane j keeps the probability of slot j
-    int id_j = 0;
-    for (int j = 0; j < topk; ++j) {
-        // best candidate of this lane: largest logit, then lowest index
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        float bex = 0.0f;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int e = lane + 32 * i;
-            if (!taken[i] && (l[i] > bv || (l[i] == bv && e < bi))) {
-                bv = l[i];
-                bi = e;
-                bex = ex[i];
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            const float oex = __shfl_xor_sync(0xffffffffu, bex, o);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-                bex = oex;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < EPL; ++i)
-            if (lane + 32 * i == bi) taken[i] = true;
-        if (lane == j) {
-            id_j = bi;
-            psel_j = __fdiv_rn(bex, sum);
-        }
-    }
-    // renormalise over the k selected, summing in slot order
-    float ssel = 0.0f;
-    for (int j = 0; j < topk; ++j) ssel = __fadd_rn(ssel, __shfl_sync(0xffffffffu, psel_j, j));
-    if (lane < topk) {
-        ids[t * topk + lane] = id_j;
-        wts[t * topk + lane] = __fdiv_rn(psel_j, ssel);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// a6: plan.  One CTA of 1024 threads.
+// a5 + a6: routing and the expert plan, one warp per token.
+//   routing: lane l holds experts l, l + 32, ... (E <= 32 * EPL); fp32 softmax
+//   with the project exponential, top-k by logit (ties to the lower expert
+//   index), weights renormalised over the k in slot order;
+//   plan: each selected (token, slot) takes its rank inside its expert from a
+//   global atomic counter (any order is a valid expert-sorted order); the last
+//   CTA to finish scans the counts into offsets, the 128-row tile offsets of
+//   the grouped GEMMs and the list of touched experts.
+// counts[E] and *done must be zero on entry.
 struct MoePlan {
     int32_t* counts;     // [E]
     int32_t* offsets;    // [E + 1]
     int32_t* active;     // [E] touched experts, ascending
     int32_t* n_active;   // [1]
     int32_t* tile_off;   // [E + 1] prefix sum of ceil(counts / 128): grouped-GEMM row tiles
-    int32_t* row_of;     // [T * topk] expert-sorted row of (token, slot)
-    int32_t* row_tok;    // [R] token of each sorted row
-    int32_t* row_slot;   // [R] slot of each sorted row
-    float* row_w;        // [R] routing weight of each sorted row
+    int32_t* rank;       // [T * topk] rank of (token, slot) inside its expert
+    int32_t* done;       // [1] finished CTAs
 };
 
-__global__ void __launch_bounds__(1024) moe_plan_kernel(const int32_t* __restrict__ ids,
-                                                        const float* __restrict__ wts, int64_t n, int E,
-                                                        int topk, MoePlan p) {
-    __shared__ int cnt[kMoeMaxExperts];
-    __shared__ int off[kMoeMaxExperts];
-    __shared__ int warp_tot[32];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-    __syncthreads();
-    // rank of each entry inside its expert (arrival order; any order is valid)
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-        const int e = ids[i];
-        p.row_of[i] = (e >= 0 && e < E) ? atomicAdd(&cnt[e], 1) : 0;   // ids come from moe_route_kernel: always < E
-    }
-    __syncthreads();
-    // exclusive scan of cnt over E <= 1024 (one element per thread)
-    const int e = threadIdx.x;
-    const int c = e < E ? cnt[e] : 0;
+template <int EPL>
+__global__ void __launch_bounds__(256) moe_route_plan_kernel(const uint16_t* __restrict__ logits, int64_t T, int E,
+                                                             int topk, int32_t* __restrict__ ids,
+                                                             float* __restrict__ wts, MoePlan p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = c;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t < T) {
+        float l[EPL], ex[EPL];
+        bool taken[EPL];
+        float mx = -INFINITY;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_tot[lane];
-        int wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += v;
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            l[i] = e < E ? bf16_bits_to_float(logits[t * E + e]) : -INFINITY;
+            if (isnan(l[i])) l[i] = -INFINITY;   // out of domain; keeps the selection well defined
+            taken[i] = e >= E;
+            mx = fmaxf(mx, l[i]);
         }
-        warp_tot[lane] = wi - w;   // exclusive prefix of warp totals
-    }
-    __syncthreads();
-    const int excl = incl - c + warp_tot[warp];
-    if (e < E) {
-        off[e] = excl;
-        p.counts[e] = c;
-        p.offsets[e] = excl;
-        if (e == E - 1) p.offsets[E] = excl + c;
-    }
-    // compact list of touched experts: rank among experts with c > 0
-    const unsigned ball = __ballot_sync(0xffffffffu, c > 0);
-    __syncthreads();
-    if (lane == 0) warp_tot[warp] = __popc(ball);
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_tot[lane];
-        int wi = w;
+        mx = warp_max(mx);
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += v;
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            ex[i] = e < E ? exp_proj(__fsub_rn(l[i], mx)) : 0.0f;
         }
-        warp_tot[lane] = wi - w;
-        if (lane == 31) p.n_active[0] = wi;
+        // softmax denominator summed in expert-index order, as a serial loop
+        // would: stage the exponentials, one lane folds them, then broadcast
+        __shared__ float ex_s[8][32 * EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) ex_s[warp][lane + 32 * i] = ex[i];
+        __syncwarp();
+        float sum = 0.0f;
+        if (lane == 0)
+            for (int e = 0; e < E; ++e) sum = __fadd_rn(sum, ex_s[warp][e]);
+        sum = __shfl_sync(0xffffffffu, sum, 0);
+
+        float psel_j = 0.0f;   // lane j keeps the probability of slot j
+        int id_j = 0;
+        for (int j = 0; j < topk; ++j) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            float bex = 0.0f;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = lane + 32 * i;
+                if (!taken[i] && (l[i] > bv || (l[i] == bv && e < bi))) {
+                    bv = l[i];
+                    bi = e;
+                    bex = ex[i];
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                const float oex = __shfl_xor_sync(0xffffffffu, bex, o);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                    bex = oex;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (lane + 32 * i == bi) taken[i] = true;
+            if (lane == j) {
+                id_j = bi;
+                psel_j = __fdiv_rn(bex, sum);
+            }
+        }
+        float ssel = 0.0f;
+        for (int j = 0; j < topk; ++j) ssel = __fadd_rn(ssel, __shfl_sync(0xffffffffu, psel_j, j));
+        if (lane < topk) {
+            ids[t * topk + lane] = id_j;
+            wts[t * topk + lane] = __fdiv_rn(psel_j, ssel);
+            p.rank[t * topk + lane] = atomicAdd(p.counts + id_j, 1);
+        }
     }
+
+    // ---- the last CTA scans the histogram (E <= 256: one expert per thread)
+    __shared__ int last;
+    __shared__ int warp_tot[8];
+    __threadfence();
     __syncthreads();
-    if (e < E && c > 0) p.active[warp_tot[warp] + __popc(ball & ((1u << lane) - 1u))] = e;
-    // exclusive scan of the 128-row tiles of each expert
+    if (threadIdx.x == 0) last = (atomicAdd(p.done, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const int e = threadIdx.x;
+    const int c = e < E ? __ldcg(p.counts + e) : 0;
     const int mt = (c + 127) / 128;
-    int tincl = mt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, tincl, o);
-        if (lane >= o) tincl += v;
-    }
-    __syncthreads();
-    if (lane == 31) warp_tot[warp] = tincl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_tot[lane];
-        int wi = w;
+    auto block_excl_scan = [&](int v) {   // exclusive scan over the 256 threads; returns (excl, total)
+        int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += v;
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
         }
-        warp_tot[lane] = wi - w;
-    }
-    __syncthreads();
-    if (e < E) {
-        const int texcl = tincl - mt + warp_tot[warp];
-        p.tile_off[e] = texcl;
-        if (e == E - 1) p.tile_off[E] = texcl + mt;
-    }
-    // final rows and the per-row metadata of the sorted order
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-        const int r = off[ids[i]] + p.row_of[i];
-        p.row_of[i] = r;
-        p.row_tok[r] = (int)(i / topk);
-        p.row_slot[r] = (int)(i % topk);
-        p.row_w[r] = wts[i];
-    }
+        __syncthreads();
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            if (w < warp) before += warp_tot[w];
+            total += warp_tot[w];
+        }
+        return make_int2(incl - v + before, total);
+    };
+    const int2 off = block_excl_scan(c);
+    if (e < E) p.offsets[e] = off.x;
+    if (e == 0) p.offsets[E] = off.y;
+    const int2 toff = block_excl_scan(mt);
+    if (e < E) p.tile_off[e] = toff.x;
+    if (e == 0) p.tile_off[E] = toff.y;
+    const int2 act = block_excl_scan(c > 0 ? 1 : 0);
+    if (e < E && c > 0) p.active[act.x] = e;
+    if (e == 0) p.n_active[0] = act.y;
 }
 
 // ---------------------------------------------------------------------------
 // a7: per-token quant of x, scattered to the token's sorted rows.  One CTA per
 // token with one 16-byte vector (8 bf16) per thread; blockDim is H/8 rounded
 // up to a whole number of warps (H <= 8 * 1024).
+struct MoeRows {
+    const int32_t* ids;      // [T * topk]
+    const float* wts;        // [T * topk]
+    const int32_t* rank;     // [T * topk]
+    const int32_t* offsets;  // [E + 1]
+    int32_t* row_of;         // [T * topk] sorted row of (token, slot)
+    int32_t* row_tok;        // [R]
+    int32_t* row_slot;       // [R]
+    float* row_w;            // [R]
+};
+
 __global__ void __launch_bounds__(1024) moe_quant_scatter_kernel(const uint16_t* __restrict__ x, int H, int topk,
-                                                                 const int32_t* __restrict__ row_of,
+                                                                 MoeRows rows,
                                                                  int8_t* __restrict__ xq, float* __restrict__ sxr,
-                                                                 float* __restrict__ out_f32,
+                                                                 float* __restrict__ clear_rows,
                                                                  int8_t* __restrict__ dbg_qx,
                                                                  float* __restrict__ dbg_sx) {
     const int64_t t = blockIdx.x;
+    // sorted rows of this token's slots (and their metadata)
+    __shared__ int srow[kMoeMaxTopk];
+    if (threadIdx.x < topk) {
+        const int64_t i = t * topk + threadIdx.x;
+        const int r = __ldg(rows.offsets + __ldg(rows.ids + i)) + __ldg(rows.rank + i);
+        srow[threadIdx.x] = r;
+        rows.row_of[i] = r;
+        rows.row_tok[r] = (int)t;
+        rows.row_slot[r] = threadIdx.x;
+        rows.row_w[r] = __ldg(rows.wts + i);
+    }
     const int v = threadIdx.x;          // vector index, 8 bf16
     const bool active = v < H / 8;
     float f[8];
@@ -264,16 +239,17 @@ __global__ void __launch_bounds__(1024) moe_quant_scatter_kernel(const uint16_t*
     }
     const uint2 codes = make_uint2(pk[0], pk[1]);
     for (int j = 0; j < topk; ++j) {
-        const int r = row_of[t * topk + j];
+        const int r = srow[j];
         *reinterpret_cast<uint2*>(xq + (int64_t)r * H + v * 8) = codes;
         if (threadIdx.x == 0) sxr[r] = s;
     }
     if (dbg_qx) *reinterpret_cast<uint2*>(dbg_qx + t * H + v * 8) = codes;
     if (dbg_sx && threadIdx.x == 0) dbg_sx[t] = s;
-    // clear this token's fp32 output row for the gemm2 combine
-    float4* o = reinterpret_cast<float4*>(out_f32 + t * H) + 2 * v;
-    o[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (clear_rows) {   // atomic combine: this token's fp32 output row starts at zero
+        float4* o = reinterpret_cast<float4*>(clear_rows + t * H) + 2 * v;
+        o[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -292,10 +268,13 @@ struct MoeGemmArgs {
     int rows, K;
     // gemm1: gated intermediate a [R, rows / 2] fp32
     float* a_out;
-    // gemm2: combine into out_f32 [T, rows]
+    // gemm2: w * y2 of each sorted row into contrib [T * topk, rows] at (token, slot),
+    // or (topk == 0) added atomically into contrib [T, rows]
     const int32_t* row_tok;
+    const int32_t* row_slot;
     const float* row_w;
-    float* out_f32;
+    float* contrib;
+    int topk;
 };
 
 template <int WN, int WK, int TG, bool GATED>
@@ -337,13 +316,19 @@ __global__ void __launch_bounds__(kGemvThreads) moe_gemm_kernel(MoeGemmArgs m) {
                         m.a_out[(int64_t)r * (m.rows / 2) + pair] = __fmul_rn(silu_proj(vg), vu);
                     } else {
                         const float wr = __ldg(m.row_w + r);
-                        float* orow = m.out_f32 + (int64_t)__ldg(m.row_tok + r) * m.rows;
+                        // topk > 0: store at (token, slot); 0: atomic add into the token's row
+                        const int64_t oi = m.topk > 0 ? (int64_t)__ldg(m.row_tok + r) * m.topk + __ldg(m.row_slot + r)
+                                                      : (int64_t)__ldg(m.row_tok + r);
+                        float* orow = m.contrib + oi * m.rows;
 #pragma unroll
                         for (int jr = 0; jr < 2; ++jr) {   // weight row g + 8 jr
                             const int n = block * 16 + g + 8 * jr;
                             const float y2 =
                                 __fmul_rn(__fmul_rn(__int2float_rn(acc[tg][2 * jr + jt]), sx), __ldg(swe + n));
-                            atomicAdd(orow + n, __fmul_rn(wr, y2));
+                            if (m.topk > 0)
+                                orow[n] = __fmul_rn(wr, y2);
+                            else
+                                atomicAdd(orow + n, __fmul_rn(wr, y2));
                         }
                     }
                 }
@@ -354,15 +339,25 @@ __global__ void __launch_bounds__(kGemvThreads) moe_gemm_kernel(MoeGemmArgs m) {
 }
 
 // ---------------------------------------------------------------------------
-// a11 tail: fp32 combine buffer -> bf16 output; optional debug gathers.
-__global__ void moe_finalize_kernel(const float* __restrict__ out_f32, uint16_t* __restrict__ y, int64_t n) {
+// a11: out[t, n] = bf16( sum over slots j = 0 .. k-1 of contrib[t, j, n] ),
+// summed in fp32 in slot order.  Four columns per thread (H % 4 == 0).
+// With topk == 1 this is the plain fp32 -> bf16 conversion of an
+// already-combined [T, H] buffer.
+__global__ void moe_finalize_kernel(const float* __restrict__ contrib, uint16_t* __restrict__ y, int64_t T, int H,
+                                    int topk) {
     const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (i + 3 < n) {
-        const float4 v = *reinterpret_cast<const float4*>(out_f32 + i);
-        *reinterpret_cast<uint2*>(y + i) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-    } else {
-        for (int64_t j = i; j < n; ++j) y[j] = float_to_bf16_bits(out_f32[j]);
+    if (i >= T * H) return;
+    const int64_t t = i / H, n = i % H;
+    const float* src = contrib + t * topk * H + n;
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+    for (int j = 0; j < topk; ++j) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(src + (int64_t)j * H));
+        a0 = __fadd_rn(a0, v.x);
+        a1 = __fadd_rn(a1, v.y);
+        a2 = __fadd_rn(a2, v.z);
+        a3 = __fadd_rn(a3, v.w);
     }
+    *reinterpret_cast<uint2*>(y + i) = make_uint2(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3));
 }
 
 __global__ void moe_debug_gather_kernel(const int8_t* __restrict__ qa, const float* __restrict__ sa,

@@ -143,6 +143,58 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
     }
 }
 
+// Short rows (K <= 32 lanes x 8 vectors): one warp per row, 8 rows per CTA.
+template <typename Tin>
+__global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restrict__ x, int64_t rows, int64_t K,
+                                                              int8_t* __restrict__ q, float* __restrict__ s) {
+    using VT = VecTraits<Tin>;
+    constexpr int E = VT::kElems;
+    constexpr int kMaxV = 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int64_t nvec = K / E;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+    uint4 regs[kMaxV];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxV; ++i) {
+        const int64_t v = lane + 32 * i;
+        if (v < nvec) {
+            regs[i] = __ldcg(xr + v);
+            float f[E];
+            VT::unpack(regs[i], f);
+#pragma unroll
+            for (int j = 0; j < E; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        }
+    }
+    amax = warp_max(amax);
+    const float sc = __fdiv_rn(amax, 127.0f);
+    if (lane == 0) s[row] = sc;
+    int8_t* qr = q + row * K;
+#pragma unroll
+    for (int i = 0; i < kMaxV; ++i) {
+        const int64_t v = lane + 32 * i;
+        if (v < nvec) {
+            float f[E];
+            VT::unpack(regs[i], f);
+            uint32_t packed[E / 4];
+#pragma unroll
+            for (int j = 0; j < E / 4; ++j) packed[j] = 0u;
+            if (sc != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < E; ++j)
+                    packed[j >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_code(f[j], sc) << (8 * (j & 3));
+            }
+            if constexpr (E == 8) {
+                *reinterpret_cast<uint2*>(qr + v * E) = make_uint2(packed[0], packed[1]);
+            } else {
+                *reinterpret_cast<uint32_t*>(qr + v * E) = packed[0];
+            }
+        }
+    }
+}
+
 // Picks the cluster width and launches.  Requirements (checked by callers):
 // K % (16 / sizeof(Tin)) == 0, ldx likewise, 16-byte aligned x, 8-byte aligned q rows.
 template <typename Tin>
@@ -150,6 +202,11 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
                               cudaStream_t stream, int num_sms, int* zero_buf = nullptr, int zero_n = 0) {
     constexpr int E = VecTraits<Tin>::kElems;
     const int64_t nvec = K / E;
+    if (nvec <= 256 && rows >= 4 * (int64_t)num_sms && zero_n == 0 && ldx == K && ldq == K) {
+        // many short rows (the MoE requant): a warp per row
+        quant_rows_warp_kernel<Tin><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(x, rows, K, q, s);
+        return cudaGetLastError();
+    }
     int NT = nvec <= 64 ? 64 : (nvec <= 128 ? 128 : 256);
     // smallest cluster width that fits the row in registers
     int cl = (int)((nvec + (int64_t)NT * kQuantMaxVec - 1) / ((int64_t)NT * kQuantMaxVec));

@@ -313,6 +313,8 @@ struct MoeWs {
     int32_t* active;
     int32_t* n_active;
     int32_t* tile_off;
+    int32_t* rank;
+    int32_t* done;
     int32_t* row_of;
     int32_t* row_tok;
     int32_t* row_slot;
@@ -326,6 +328,13 @@ struct MoeWs {
     size_t bytes;
 };
 
+// The combine sums each token's k contributions in slot order -- the same
+// fp32 steps as the definition -- while the [T * k, H] contribution buffer
+// fits comfortably in L2; beyond that it accumulates with fp32 vector atomics
+// into [T, H] (order unspecified).
+constexpr size_t kMoeExactCombineBytes = (size_t)64 << 20;
+inline bool moe_exact_combine(int64_t R, int H) { return (size_t)R * H * 4 <= kMoeExactCombineBytes; }
+
 MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     MoeWs w;
     const int64_t R = T * topk;
@@ -338,11 +347,14 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     };
     w.ids = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.wts = reinterpret_cast<float*>(take((size_t)R * 4));
-    w.counts = reinterpret_cast<int32_t*>(take((size_t)E * 4));
+    // counts and the CTA counter are adjacent: one memset clears both
+    w.counts = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+    w.done = w.counts + E;
     w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
     w.active = reinterpret_cast<int32_t*>(take((size_t)E * 4));
     w.n_active = reinterpret_cast<int32_t*>(take(4));
     w.tile_off = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+    w.rank = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.row_of = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.row_tok = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.row_slot = reinterpret_cast<int32_t*>(take((size_t)R * 4));
@@ -352,7 +364,8 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     w.a = reinterpret_cast<float*>(take((size_t)R * I * 4));
     w.qa = reinterpret_cast<int8_t*>(take((size_t)R * I));
     w.sa = reinterpret_cast<float*>(take((size_t)R * 4));
-    w.out = reinterpret_cast<float*>(take((size_t)T * H * 4));
+    // w * y2 at (token, slot), or the atomically combined [T, H] for large T
+    w.out = reinterpret_cast<float*>(take(moe_exact_combine(R, H) ? (size_t)R * H * 4 : (size_t)T * H * 4));
     w.bytes = o;
     return w;
 }
@@ -361,9 +374,9 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
 // [R, K], B = the experts' weights viewed as [E * N, K].
 template <int EPI>
 int launch_tc_grouped(const int8_t* A, int64_t rowsA, const int8_t* B, int E, TcParams p, cudaStream_t st) {
-    constexpr int BN = 256, STAGES = 4;
+    constexpr int BN = 256, STAGES = 4, NEPI = 8;
     using SM = TcSmem<BN, STAGES>;
-    auto kern = gemm_i8_tc_kernel<BN, STAGES, EPI, 2, true>;
+    auto kern = gemm_i8_tc_kernel<BN, STAGES, EPI, 2, true, NEPI>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
@@ -380,7 +393,7 @@ int launch_tc_grouped(const int8_t* A, int64_t rowsA, const int8_t* B, int E, Tc
     p.num_m_tiles = 0;
     p.num_n_tiles = (p.N + BN - 1) / BN;
     p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
-    kern<<<device_sms(dev), kTcThreads, SM::kBytes, st>>>(ta, tb, p);
+    kern<<<device_sms(dev), tc_threads<NEPI>(), SM::kBytes, st>>>(ta, tb, p);
     return last_launch_status();
 }
 
@@ -576,15 +589,16 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     const int64_t R = T * topk;
     int rc;
 
-    moe_route_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts);
+    if (cudaMemsetAsync(w.counts, 0, (size_t)(E + 1) * 4, st) != cudaSuccess) return W8A8_ERR_CUDA;
+    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.rank, w.done};
+    moe_route_plan_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts, plan);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
-    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.row_of, w.row_tok, w.row_slot, w.row_w};
-    moe_plan_kernel<<<1, 1024, 0, st>>>(w.ids, w.wts, R, E, topk, plan);
-    if ((rc = last_launch_status()) != W8A8_OK) return rc;
-
+    const bool exact_combine = moe_exact_combine(R, H);
+    MoeRows rows = {w.ids, w.wts, w.rank, w.offsets, w.row_of, w.row_tok, w.row_slot, w.row_w};
     moe_quant_scatter_kernel<<<(unsigned)T, (unsigned)((H / 8 + 31) / 32 * 32), 0, st>>>(
-        x, H, topk, w.row_of, w.xq, w.sxr, w.out, dbg ? dbg->qx : nullptr, dbg ? dbg->sx : nullptr);
+        x, H, topk, rows, w.xq, w.sxr, exact_combine ? nullptr : w.out, dbg ? dbg->qx : nullptr,
+        dbg ? dbg->sx : nullptr);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
     const int max_active = (int)(R < E ? R : E);
@@ -615,9 +629,13 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
         p2.offsets = w.offsets;
         p2.tile_off = w.tile_off;
         p2.row_tok = w.row_tok;
+        p2.row_slot = w.row_slot;
         p2.row_w = w.row_w;
-        p2.out_f32 = w.out;
-        if ((rc = launch_tc_grouped<kEpiMoeCombine>(w.qa, R, w2, E, p2, st)) != W8A8_OK) return rc;
+        p2.contrib = w.out;
+        p2.topk = topk;
+        rc = exact_combine ? launch_tc_grouped<kEpiMoeCombine>(w.qa, R, w2, E, p2, st)
+                           : launch_tc_grouped<kEpiMoeCombineAtomic>(w.qa, R, w2, E, p2, st);
+        if (rc != W8A8_OK) return rc;
     }
     MoeGemmArgs g1 = {};
     g1.w = w13;
@@ -651,15 +669,17 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     g2.rows = H;
     g2.K = I;
     g2.row_tok = w.row_tok;
+    g2.row_slot = w.row_slot;
     g2.row_w = w.row_w;
-    g2.out_f32 = w.out;
+    g2.contrib = w.out;
+    g2.topk = exact_combine ? topk : 0;
     rc = wide ? launch_moe_gemm<8, 1, 4, false>(g2, H / 128, max_active, st)
               : launch_moe_gemm<8, 1, 1, false>(g2, H / 128, max_active, st);
     if (rc != W8A8_OK) return rc;
     }
 
     const int64_t n = T * H;
-    moe_finalize_kernel<<<(unsigned)((n / 4 + 255) / 256 + 1), 256, 0, st>>>(w.out, y, n);
+    moe_finalize_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, st>>>(w.out, y, T, H, exact_combine ? topk : 1);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
     if (dbg) {

@@ -1,7 +1,9 @@
 """GPU parity of the routed W8A8 MoE layer (a5 .. a11) against the CPU
-oracle: expert ids, histogram, x codes and the gated intermediate's codes
-and scales bit for bit; routing weights to fp32 rounding; the bf16 output
-within one bf16 ulp plus the reassociation bound of the fp32 combine."""
+oracle: expert ids, histogram, routing weights, x codes, the gated
+intermediate's codes and scales bit for bit; the bf16 output bit for bit
+while the slot-order combine is used (the kernels take the oracle's fp32
+steps in the oracle's order), and for the large-T atomic combine within one
+bf16 ulp plus the bound on reordering a sum of k fp32 terms."""
 import numpy as np
 import pytest
 import torch
@@ -40,13 +42,19 @@ def _compare(orc, xb, lb, gpu_w, orc_w, topk, tokens):
     ref = orc.moe_forward(xb, lb, *orc_w, topk, tokens=tokens)
     t = ref["tokens"]
     assert np.array_equal(dbg["topk_ids"].cpu().numpy()[t], ref["ids"])
-    assert np.allclose(dbg["topk_w"].cpu().numpy()[t], ref["wts"], rtol=8 * 2.0 ** -24, atol=0)
+    assert np.array_equal(dbg["topk_w"].cpu().numpy()[t].view(np.uint32), ref["wts"].view(np.uint32))
     assert np.array_equal(dbg["qx"].cpu().numpy()[t], ref["qx"])
     assert np.array_equal(dbg["sx"].cpu().numpy()[t].view(np.uint32), ref["sx"].view(np.uint32))
     assert np.array_equal(dbg["qa"].cpu().numpy()[t], ref["qa"])
     assert np.array_equal(dbg["sa"].cpu().numpy()[t].view(np.uint32), ref["sa"].view(np.uint32))
-    # the k fp32 contributions may be added in any order
-    assert_bf16_close(y[t], ref["y32"], extra=2.0 ** -18 * ref["yabs"].astype(np.float64), what="moe y")
+    H = xb.shape[1]
+    if xb.shape[0] * topk * H * 4 <= 64 << 20:
+        # slot-order combine: the oracle's fp32 steps exactly
+        assert assert_bf16_close(y[t], ref["y32"], what="moe y") == 1.0
+        assert np.array_equal(y[t], ref["y"])
+    else:
+        # large T: fp32 atomics, the k contributions added in some order
+        assert_bf16_close(y[t], ref["y32"], extra=2.0 ** -18 * ref["yabs"].astype(np.float64), what="moe y")
 
 
 def _small(seed, T, E, H, I, skew=None):
