@@ -239,6 +239,23 @@ __device__ __forceinline__ int quant_code(float v, float s) {
     return max(-127, min(127, q));
 }
 
+// The same code, with rcp = __frcp_rn(s) computed once per row: y = v * rcp
+// (one rounding) differs from the correctly rounded v / s by less than
+// 2.3e-5 for |v / s| <= 127.5, so rounding y to the nearest integer gives
+// rne(v / s) unless y lies within 2^-14 of a half-integer; only then (about
+// one element in 8000) is the exact division taken.
+__device__ __forceinline__ int quant_code_rcp(float v, float s, float rcp) {
+    const float y = __fmul_rn(v, rcp);
+    const float fl = floorf(y);
+    const float d = __fsub_rn(__fsub_rn(y, fl), 0.5f);   // exact: distance of y above fl + 1/2
+    int q;
+    if (fabsf(d) <= 6.103515625e-05f || !(fabsf(rcp) < 1.0e38f))
+        q = __float2int_rn(__fdiv_rn(v, s));
+    else
+        q = (int)fl + (d > 0.0f ? 1 : 0);
+    return max(-127, min(127, q));
+}
+
 // Four fp32 atomic adds in one vector reduction (16-byte aligned address).
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)

@@ -67,8 +67,9 @@ __global__ void __launch_bounds__(256) fwht128_quant_kernel(const uint16_t* __re
     const float sf = bf16_bits_to_float(sb);
     uint32_t pk = 0u;
     if (sf != 0.0f) {
+        const float rcp = __frcp_rn(sf);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) pk |= (uint32_t)(uint8_t)(int8_t)quant_code(v[j], sf) << (8 * j);
+        for (int j = 0; j < 4; ++j) pk |= (uint32_t)(uint8_t)(int8_t)quant_code_rcp(v[j], sf, rcp) << (8 * j);
     }
     *reinterpret_cast<uint32_t*>(q + m * K + g * 128 + 4 * lane) = pk;
     if (lane == 0) s[m * G + g] = sb;

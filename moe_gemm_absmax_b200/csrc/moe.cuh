@@ -234,8 +234,10 @@ __global__ void __launch_bounds__(1024) moe_quant_scatter_kernel(const uint16_t*
     if (!active) return;
     uint32_t pk[2] = {0u, 0u};
     if (s != 0.0f) {
+        const float rcp = __frcp_rn(s);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) pk[j >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_code(f[j], s) << (8 * (j & 3));
+        for (int j = 0; j < 8; ++j)
+            pk[j >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_code_rcp(f[j], s, rcp) << (8 * (j & 3));
     }
     const uint2 codes = make_uint2(pk[0], pk[1]);
     for (int j = 0; j < topk; ++j) {

@@ -56,7 +56,7 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // grid = (CL * rows); cluster = (CL, 1, 1).  Cluster r handles row r; its
 // CTA c handles vectors [c * vpc, (c + 1) * vpc) (vpc = vectors per CTA).
-template <typename Tin, int NT>
+template <typename Tin, int NT, int MAXV = kQuantMaxVec>
 __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ x, int64_t K, int64_t ldx,
                                                         int8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
                                                         int vpc, int cl, int* zero_buf, int zero_n) {
@@ -75,10 +75,10 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
     const int64_t v1 = min(nvec, v0 + vpc);
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
 
-    uint4 regs[kQuantMaxVec];
+    uint4 regs[MAXV];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kQuantMaxVec; ++i) {
+    for (int i = 0; i < MAXV; ++i) {
         const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
         if (v < v1) {
             regs[i] = __ldg(xr + v);
@@ -115,11 +115,12 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
     __syncthreads();
     amax = red[0];
     const float sc = __fdiv_rn(amax, 127.0f);
+    const float rcp = __frcp_rn(sc);
     if (crank == 0 && threadIdx.x == 0) s[row] = sc;
 
     int8_t* qr = q + row * ldq;
 #pragma unroll
-    for (int i = 0; i < kQuantMaxVec; ++i) {
+    for (int i = 0; i < MAXV; ++i) {
         const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
         if (v < v1) {
             float f[E];
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
             if (sc != 0.0f) {
 #pragma unroll
                 for (int j = 0; j < E; ++j) {
-                    const uint32_t b = (uint32_t)(uint8_t)(int8_t)quant_code(f[j], sc);
+                    const uint32_t b = (uint32_t)(uint8_t)(int8_t)quant_code_rcp(f[j], sc, rcp);
                     packed[j >> 2] |= b << (8 * (j & 3));
                 }
             }
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
     }
     amax = warp_max(amax);
     const float sc = __fdiv_rn(amax, 127.0f);
+    const float rcp = __frcp_rn(sc);
     if (lane == 0) s[row] = sc;
     int8_t* qr = q + row * K;
 #pragma unroll
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
             if (sc != 0.0f) {
 #pragma unroll
                 for (int j = 0; j < E; ++j)
-                    packed[j >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_code(f[j], sc) << (8 * (j & 3));
+                    packed[j >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_code_rcp(f[j], sc, rcp) << (8 * (j & 3));
             }
             if constexpr (E == 8) {
                 *reinterpret_cast<uint2*>(qr + v * E) = make_uint2(packed[0], packed[1]);
@@ -195,8 +197,13 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
     }
 }
 
-// Picks the cluster width and launches.  Requirements (checked by callers):
-// K % (16 / sizeof(Tin)) == 0, ldx likewise, 16-byte aligned x, 8-byte aligned q rows.
+// Picks the CTA size, the cluster width and the register slice, and launches.
+// Requirements (checked by callers): K % (16 / sizeof(Tin)) == 0, ldx likewise,
+// 16-byte aligned x, 8-byte aligned q rows.
+//   many rows: one CTA per row (no cluster), 64..1024 threads so that each
+//              thread holds at most 4 vectors where possible;
+//   few rows (decode): a power-of-two cluster of up to 8 CTAs per row, so that
+//              more SMs pull the row from HBM.
 template <typename Tin>
 cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* s,
                               cudaStream_t stream, int num_sms, int* zero_buf = nullptr, int zero_n = 0) {
@@ -207,14 +214,21 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
         quant_rows_warp_kernel<Tin><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(x, rows, K, q, s);
         return cudaGetLastError();
     }
-    int NT = nvec <= 64 ? 64 : (nvec <= 128 ? 128 : 256);
-    // smallest cluster width that fits the row in registers
-    int cl = (int)((nvec + (int64_t)NT * kQuantMaxVec - 1) / ((int64_t)NT * kQuantMaxVec));
-    if (cl < 1) cl = 1;
-    // few rows: widen the cluster so that more SMs pull the row from HBM
-    while (cl < 8 && rows * cl < 2 * num_sms && nvec / (cl * 2) >= (int64_t)NT) cl *= 2;
-    if (cl > 8) return cudaErrorInvalidValue;
-    int vpc = (int)((nvec + cl - 1) / cl);
+    int NT, cl;
+    if (rows >= 2 * (int64_t)num_sms && nvec <= 1024 * 6) {
+        // (1024 threads leave 64 registers a thread: at most 6 vectors)
+        cl = 1;
+        NT = 64;
+        while (NT < 1024 && nvec > (int64_t)NT * 4) NT *= 2;
+    } else {
+        NT = nvec <= 64 ? 64 : (nvec <= 128 ? 128 : 256);
+        cl = 1;
+        while (cl < 8 && nvec > (int64_t)NT * 4 * cl) cl *= 2;                       // fit in 4 / thread
+        if (nvec > (int64_t)NT * kQuantMaxVec * cl) return cudaErrorInvalidValue;
+        while (cl < 8 && rows * cl < 2 * num_sms && nvec / (cl * 2) >= (int64_t)NT) cl *= 2;   // spread
+    }
+    const int vpc = (int)((nvec + cl - 1) / cl);
+    const int per_thread = (vpc + NT - 1) / NT;
 
     cudaLaunchConfig_t cfg = {};
     if (rows * cl > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -228,15 +242,27 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = cl > 1 ? 1 : 0;
+#define W8A8_QUANT_LAUNCH(nt, mv) \
+    return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, nt, mv>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n)
     switch (NT) {
         case 64:
-            return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, 64>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n);
+            if (per_thread <= 4) W8A8_QUANT_LAUNCH(64, 4);
+            W8A8_QUANT_LAUNCH(64, 16);
         case 128:
-            return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, 128>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n);
+            if (per_thread <= 4) W8A8_QUANT_LAUNCH(128, 4);
+            W8A8_QUANT_LAUNCH(128, 16);
+        case 256:
+            if (per_thread <= 4) W8A8_QUANT_LAUNCH(256, 4);
+            if (per_thread <= 8) W8A8_QUANT_LAUNCH(256, 8);
+            W8A8_QUANT_LAUNCH(256, 16);
+        case 512:
+            W8A8_QUANT_LAUNCH(512, 4);
         default:
-            return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, 256>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n);
+            if (per_thread <= 4) W8A8_QUANT_LAUNCH(1024, 4);
+            W8A8_QUANT_LAUNCH(1024, 6);
     }
+#undef W8A8_QUANT_LAUNCH
 }
 
 }  // namespace w8a8

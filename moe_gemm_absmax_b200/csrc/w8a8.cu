@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "fwht.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
 #include "moe.cuh"
@@ -106,6 +107,45 @@ int launch_tc(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     return last_launch_status();
 }
 
+// Pair-tile GEMM (cta_group::2, 256 x 256 tiles over two SMs).
+template <int EPI>
+int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
+    auto kern = gemm_i8_tc2_kernel<EPI>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    static int max_clusters[kMaxDevices] = {0};
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kTc2Threads, 1, 1);
+    cfg.dynamicSmemBytes = Tc2Smem::kBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (max_clusters[dev] == 0) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Smem::kBytes) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        cfg.gridDim = dim3((unsigned)(2 * (device_sms(dev) / 2)), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_sms(dev) / 2;
+        max_clusters[dev] = n;
+    }
+    CUtensorMap ta, tb;
+    if (!make_tmap_i8(&ta, A, (uint64_t)p.M, (uint64_t)p.K, 128)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tb, B, (uint64_t)p.N, (uint64_t)p.K, 128)) return W8A8_ERR_CUDA;
+    p.num_m_tiles = (p.M + kTc2BM - 1) / kTc2BM;
+    p.num_n_tiles = (p.N + kTc2BN - 1) / kTc2BN;
+    p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
+    const int tiles = p.num_m_tiles * p.num_n_tiles;
+    const int clusters = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, p));
+}
+
 // Tile width: the one with less work in its last wave (256 on ties).
 int pick_bn(int64_t M, int64_t N, int sms) {
     const int64_t mt = (M + kTcBM - 1) / kTcBM;
@@ -113,6 +153,9 @@ int pick_bn(int64_t M, int64_t N, int sms) {
     const int64_t w128 = (mt * ((N + 127) / 128) + sms - 1) / sms;
     return (w128 * 128 < w256 * 256) ? 128 : 256;
 }
+
+// Token counts from which the pair-tile kernel is used.
+constexpr int64_t kTc2MinM = 256;
 
 int run_tc(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M, int64_t N,
            int64_t K, int epi, cudaStream_t st) {
@@ -123,6 +166,7 @@ int run_tc(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw,
     p.sx = sx;
     p.sw = sw;
     p.out = out;
+    if (M >= kTc2MinM) return epi == kEpiBf16 ? launch_tc2<kEpiBf16>(qx, qw, p, st) : launch_tc2<kEpiS32>(qx, qw, p, st);
     const int bn = pick_bn(M, N, current_sms());
     if (epi == kEpiBf16)
         return bn == 256 ? launch_tc<256, 4, kEpiBf16, 2>(qx, qw, p, st) : launch_tc<128, 6, kEpiBf16, 2>(qx, qw, p, st);

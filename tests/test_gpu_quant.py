@@ -60,3 +60,21 @@ def test_exp_proj_bit_exact(orc):
     x = np.concatenate([x, np.float32([88.0, -87.0, 100.0, -100.0, 0.0, -0.0])])
     y = w8a8.exp_proj(torch.from_numpy(x).cuda()).cpu().numpy()
     assert np.array_equal(y.view(np.uint32), orc.exp_proj(x).view(np.uint32))
+
+
+def test_quant_near_ties_take_the_exact_path(orc):
+    """Values a few ulps from a half-integer multiple of the scale: the
+    reciprocal-multiply fast path must hand them to the exact division."""
+    rng = np.random.default_rng(11)
+    rows = []
+    for scale in (1 / 16, 0.0123, 3.7e-3):
+        n = rng.integers(-126, 126, 256).astype(np.float64)
+        eps = rng.choice([0.0, 2.0 ** -23, -(2.0 ** -23), 2.0 ** -20, -(2.0 ** -20), 2.0 ** -15, -(2.0 ** -15)], 256)
+        v = ((n + 0.5) * (1.0 + eps) * scale).astype(np.float32)
+        v[0] = np.float32(127 * scale)            # fixes absmax, hence s = fp32(127 scale / 127)
+        rows.append(v)
+    w = np.stack(rows)
+    q, s = w8a8.quant_rows_f32(torch.from_numpy(w).cuda())
+    qo, so = orc.quant_rows_f32(w)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
