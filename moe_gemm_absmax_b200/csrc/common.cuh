@@ -244,16 +244,136 @@ __device__ __forceinline__ int quant_code(float v, float s) {
 // 2.3e-5 for |v / s| <= 127.5, so rounding y to the nearest integer gives
 // rne(v / s) unless y lies within 2^-14 of a half-integer; only then (about
 // one element in 8000) is the exact division taken.
+//
+// Rounding y: t = y + 1.5 * 2^23 lies in [2^23, 2^24), where the spacing of
+// floats is 1, so the addition itself rounds y to the nearest integer (ties
+// to even, as 1.5 * 2^23 is even) and leaves it in the low mantissa bits:
+// the code is bits(t) - bits(1.5 * 2^23).  r = t - 1.5 * 2^23 is that integer
+// as a float and e = y - r is exact (Sterbenz), so |e| says how close y is to
+// a tie.  A NaN y fails the test and takes the exact path as well.  Needs
+// |v / s| < 2^22, which holds wherever s is the row maximum of |v| over 127
+// (every caller: |v / s| <= 127.5 there).
 __device__ __forceinline__ int quant_code_rcp(float v, float s, float rcp) {
     const float y = __fmul_rn(v, rcp);
-    const float fl = floorf(y);
-    const float d = __fsub_rn(__fsub_rn(y, fl), 0.5f);   // exact: distance of y above fl + 1/2
+    const float t = __fadd_rn(y, 12582912.0f);
+    const float e = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
     int q;
-    if (fabsf(d) <= 6.103515625e-05f || !(fabsf(rcp) < 1.0e38f))
+    if (!(fabsf(e) < 0.49993896484375f) || !(fabsf(rcp) < 1.0e38f))   // 0.5 - 2^-14
         q = __float2int_rn(__fdiv_rn(v, s));
     else
-        q = (int)fl + (d > 0.0f ? 1 : 0);
+        q = (int)(__float_as_uint(t) - 0x4B400000u);
     return max(-127, min(127, q));
+}
+
+// Low bytes of four codes packed little-endian into one word.
+__device__ __forceinline__ uint32_t pack4_s8(int q0, int q1, int q2, int q3) {
+    const uint32_t lo = __byte_perm((uint32_t)q0, (uint32_t)q1, 0x0040);
+    const uint32_t hi = __byte_perm((uint32_t)q2, (uint32_t)q3, 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
+}
+
+// ---- paired fp32 arithmetic: sm_100 adds, subtracts and multiplies the two
+// fp32 halves of a 64-bit register pair in one instruction (each half
+// rounded to nearest even, as the scalar operation would be).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t d, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(d));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// max that returns NaN if either input is NaN
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// Per-row quantizer: the scale s = amax / 127, its rounded reciprocal, and
+// whether the reciprocal path applies (s normal enough that 1 / s is finite).
+struct QuantRow {
+    float s, rcp;
+    uint64_t rcp2;
+    bool zero, fast;
+    __device__ __forceinline__ explicit QuantRow(float amax) {
+        s = __fdiv_rn(amax, 127.0f);
+        rcp = __frcp_rn(s);
+        rcp2 = f2_pack(rcp, rcp);
+        zero = s == 0.0f;
+        fast = fabsf(s) < INFINITY && fabsf(rcp) < 1.0e38f;
+    }
+};
+
+// Codes of 4W consecutive values v (|v| <= 127.25 s) under row quantizer r,
+// four to a word, little-endian.  Fast path, two values per instruction:
+// y = v * rcp; t = y + 1.5 * 2^23 rounds y to the nearest integer (ties to
+// even) into the low mantissa bits of t, whose low byte is then the int8
+// code itself (|rne(y)| <= 127 here); e = y - (t - 1.5 * 2^23) is exact and
+// measures the distance from y to a tie.  y differs from v / s by < 2.3e-5,
+// so unless some |e| of the group reaches 0.5 - 2^-14 (or is NaN) the codes
+// equal clamp(rne(v / s)); otherwise the group is redone by exact division.
+template <int W>
+__device__ __forceinline__ void quant_codes(const float (&v)[4 * W], const QuantRow& r, uint32_t (&out)[W]) {
+    if (r.zero) {
+#pragma unroll
+        for (int j = 0; j < W; ++j) out[j] = 0u;
+        return;
+    }
+    bool ok = r.fast;
+    if (ok) {
+        const uint64_t magic2 = 0x4B4000004B400000ull;   // (1.5 * 2^23, 1.5 * 2^23)
+        float emax = 0.0f;
+        uint32_t tb[4 * W];
+#pragma unroll
+        for (int i = 0; i < 2 * W; ++i) {
+            const uint64_t y = f2_mul(f2_pack(v[2 * i], v[2 * i + 1]), r.rcp2);
+            const uint64_t t = f2_add(y, magic2);
+            const uint64_t e = f2_sub(y, f2_sub(t, magic2));
+            float e0, e1, t0, t1;
+            f2_unpack(e, e0, e1);
+            f2_unpack(t, t0, t1);
+            emax = fmax_nan(emax, fmax_nan(fabsf(e0), fabsf(e1)));
+            tb[2 * i] = __float_as_uint(t0);
+            tb[2 * i + 1] = __float_as_uint(t1);
+        }
+        ok = emax < 0.49993896484375f;
+        if (ok) {
+#pragma unroll
+            for (int j = 0; j < W; ++j)
+                out[j] = __byte_perm(__byte_perm(tb[4 * j], tb[4 * j + 1], 0x0040),
+                                     __byte_perm(tb[4 * j + 2], tb[4 * j + 3], 0x0040), 0x5410);
+        }
+    }
+    if (!ok) {
+#pragma unroll
+        for (int j = 0; j < W; ++j)
+            out[j] = pack4_s8(quant_code(v[4 * j], r.s), quant_code(v[4 * j + 1], r.s), quant_code(v[4 * j + 2], r.s),
+                              quant_code(v[4 * j + 3], r.s));
+    }
+}
+
+// running max of |bf16| over packed pairs: (bits & 0x7fff) orders like |value|
+// for every non-NaN bf16, and a NaN shows up as a pattern above 0x7f80
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // Four fp32 atomic adds in one vector reduction (16-byte aligned address).

@@ -22,12 +22,18 @@ namespace w8a8 {
 namespace cg = cooperative_groups;
 
 constexpr int kQuantMaxVec = 16;   // 16-byte vectors kept in registers per thread
+constexpr int64_t kQuantSmemRowMax = 200 * 1024;   // largest row staged in shared memory
 
+// Per input type: unpacking a 16-byte vector to fp32, and a running |v|
+// maximum (Acc) whose final value equals the fp32 maximum that skips NaN;
+// acc_final returns false when the fast accumulator cannot say (bf16 NaN
+// seen), and the caller then takes the fp32 maximum of its vectors itself.
 template <typename Tin>
 struct VecTraits;
 template <>
 struct VecTraits<uint16_t> {   // bf16 bits: 8 per 16 bytes
     static constexpr int kElems = 8;
+    using Acc = uint32_t;       // two 16-bit maxima of (bits & 0x7fff)
     __device__ static void unpack(const uint4& v, float (&f)[8]) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -36,22 +42,125 @@ struct VecTraits<uint16_t> {   // bf16 bits: 8 per 16 bytes
             f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
     }
+    __device__ static Acc acc_init() { return 0u; }
+    __device__ static void acc(Acc& a, const uint4& v) {
+        a = max_u16x2(a, v.x & 0x7fff7fffu);
+        a = max_u16x2(a, v.y & 0x7fff7fffu);
+        a = max_u16x2(a, v.z & 0x7fff7fffu);
+        a = max_u16x2(a, v.w & 0x7fff7fffu);
+    }
+    __device__ static bool acc_final(Acc a, float& amax) {
+        const uint32_t m = max(a & 0xffffu, a >> 16);
+        amax = __uint_as_float(m << 16);
+        return m <= 0x7f80u;
+    }
 };
 template <>
 struct VecTraits<float> {      // fp32: 4 per 16 bytes
     static constexpr int kElems = 4;
+    using Acc = float;
     __device__ static void unpack(const uint4& v, float (&f)[4]) {
         f[0] = __uint_as_float(v.x);
         f[1] = __uint_as_float(v.y);
         f[2] = __uint_as_float(v.z);
         f[3] = __uint_as_float(v.w);
     }
+    __device__ static Acc acc_init() { return 0.0f; }
+    __device__ static void acc(Acc& a, const uint4& v) {
+        a = fmaxf(a, fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))));
+        a = fmaxf(a, fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
+    }
+    __device__ static bool acc_final(Acc a, float& amax) {
+        amax = a;
+        return true;
+    }
 };
+
+// fp32 maximum of |v| over one vector, NaN skipped (fmaxf returns the other operand)
+template <typename Tin>
+__device__ __forceinline__ float vec_absmax(const uint4& raw) {
+    using VT = VecTraits<Tin>;
+    float f[VT::kElems];
+    VT::unpack(raw, f);
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VT::kElems; ++j) m = fmaxf(m, fabsf(f[j]));
+    return m;
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
+}
+
+template <int E>
+__device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&packed)[E / 4]) {
+    if constexpr (E == 8) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    } else {
+        *reinterpret_cast<uint32_t*>(dst) = packed[0];
+    }
+}
+
+// unpack one vector and write its codes
+template <typename Tin>
+__device__ __forceinline__ void quant_vec_store(const uint4& raw, const QuantRow& r, int8_t* dst) {
+    using VT = VecTraits<Tin>;
+    constexpr int E = VT::kElems;
+    float f[E];
+    VT::unpack(raw, f);
+    uint32_t packed[E / 4];
+    quant_codes<E / 4>(f, r, packed);
+    store_codes<E>(dst, packed);
+}
+
+__device__ __forceinline__ void cp_async_16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+
+// Many rows: one CTA per row, the row staged in shared memory by 16-byte
+// asynchronous copies (no registers held while the loads are in flight, so
+// an SM keeps as many rows in flight as its shared memory holds).  Each
+// thread reads back only the vectors it copied itself, so its own
+// cp.async.wait_group is the only wait before the first pass.
+template <typename Tin, int NT>
+__global__ void __launch_bounds__(NT) quant_rows_smem_kernel(const Tin* __restrict__ x, int64_t K, int64_t ldx,
+                                                             int8_t* __restrict__ q, int64_t ldq,
+                                                             float* __restrict__ s, int* zero_buf, int zero_n) {
+    using VT = VecTraits<Tin>;
+    constexpr int E = VT::kElems;
+    extern __shared__ __align__(16) uint4 row_s[];
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int64_t row = blockIdx.x;
+    const int nvec = (int)(K / E);
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
+    for (int v = threadIdx.x; v < nvec; v += NT) cp_async_16(row_s + v, xr + v);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int i = blockIdx.x * NT + threadIdx.x; i < zero_n; i += gridDim.x * NT) zero_buf[i] = 0;
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+    typename VT::Acc acc = VT::acc_init();
+    for (int v = threadIdx.x; v < nvec; v += NT) VT::acc(acc, row_s[v]);
+    float amax;
+    if (!VT::acc_final(acc, amax)) {   // NaN among this thread's values
+        amax = 0.0f;
+        for (int v = threadIdx.x; v < nvec; v += NT) amax = fmaxf(amax, vec_absmax<Tin>(row_s[v]));
+    }
+    __shared__ float red[NT / 32];
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, red[w]);
+    const QuantRow qrow(amax);
+    if (threadIdx.x == 0) s[row] = qrow.s;
+
+    int8_t* qr = q + row * ldq;
+    for (int v = threadIdx.x; v < nvec; v += NT) quant_vec_store<Tin>(row_s[v], qrow, qr + (int64_t)v * E);
 }
 
 // grid = (CL * rows); cluster = (CL, 1, 1).  Cluster r handles row r; its
@@ -76,17 +185,21 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
 
     uint4 regs[MAXV];
-    float amax = 0.0f;
+    typename VT::Acc acc = VT::acc_init();
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
         const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
         if (v < v1) {
             regs[i] = __ldg(xr + v);
-            float f[E];
-            VT::unpack(regs[i], f);
-#pragma unroll
-            for (int j = 0; j < E; ++j) amax = fmaxf(amax, fabsf(f[j]));
+            VT::acc(acc, regs[i]);
         }
+    }
+    float amax;
+    if (!VT::acc_final(acc, amax)) {   // NaN among this thread's values
+        amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i)
+            if (v0 + threadIdx.x + (int64_t)i * NT < v1) amax = fmaxf(amax, vec_absmax<Tin>(regs[i]));
     }
     __shared__ float red[NT / 32];
     __shared__ float cta_max;
@@ -113,34 +226,14 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
         if (threadIdx.x == 0) red[0] = cta_max;
     }
     __syncthreads();
-    amax = red[0];
-    const float sc = __fdiv_rn(amax, 127.0f);
-    const float rcp = __frcp_rn(sc);
-    if (crank == 0 && threadIdx.x == 0) s[row] = sc;
+    const QuantRow qrow(red[0]);
+    if (crank == 0 && threadIdx.x == 0) s[row] = qrow.s;
 
     int8_t* qr = q + row * ldq;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
         const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
-        if (v < v1) {
-            float f[E];
-            VT::unpack(regs[i], f);
-            uint32_t packed[E / 4];
-#pragma unroll
-            for (int j = 0; j < E / 4; ++j) packed[j] = 0u;
-            if (sc != 0.0f) {
-#pragma unroll
-                for (int j = 0; j < E; ++j) {
-                    const uint32_t b = (uint32_t)(uint8_t)(int8_t)quant_code_rcp(f[j], sc, rcp);
-                    packed[j >> 2] |= b << (8 * (j & 3));
-                }
-            }
-            if constexpr (E == 8) {
-                *reinterpret_cast<uint2*>(qr + v * E) = make_uint2(packed[0], packed[1]);
-            } else {
-                *reinterpret_cast<uint32_t*>(qr + v * E) = packed[0];
-            }
-        }
+        if (v < v1) quant_vec_store<Tin>(regs[i], qrow, qr + v * E);
     }
 }
 
@@ -157,43 +250,29 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
     const int64_t nvec = K / E;
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
     uint4 regs[kMaxV];
-    float amax = 0.0f;
+    typename VT::Acc acc = VT::acc_init();
 #pragma unroll
     for (int i = 0; i < kMaxV; ++i) {
         const int64_t v = lane + 32 * i;
         if (v < nvec) {
             regs[i] = __ldcg(xr + v);
-            float f[E];
-            VT::unpack(regs[i], f);
-#pragma unroll
-            for (int j = 0; j < E; ++j) amax = fmaxf(amax, fabsf(f[j]));
+            VT::acc(acc, regs[i]);
         }
     }
-    amax = warp_max(amax);
-    const float sc = __fdiv_rn(amax, 127.0f);
-    const float rcp = __frcp_rn(sc);
-    if (lane == 0) s[row] = sc;
+    float amax;
+    if (!VT::acc_final(acc, amax)) {   // NaN among this lane's values
+        amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kMaxV; ++i)
+            if (lane + 32 * i < nvec) amax = fmaxf(amax, vec_absmax<Tin>(regs[i]));
+    }
+    const QuantRow qrow(warp_max(amax));
+    if (lane == 0) s[row] = qrow.s;
     int8_t* qr = q + row * K;
 #pragma unroll
     for (int i = 0; i < kMaxV; ++i) {
         const int64_t v = lane + 32 * i;
-        if (v < nvec) {
-            float f[E];
-            VT::unpack(regs[i], f);
-            uint32_t packed[E / 4];
-#pragma unroll
-            for (int j = 0; j < E / 4; ++j) packed[j] = 0u;
-            if (sc != 0.0f) {
-#pragma unroll
-                for (int j = 0; j < E; ++j)
-                    packed[j >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_code_rcp(f[j], sc, rcp) << (8 * (j & 3));
-            }
-            if constexpr (E == 8) {
-                *reinterpret_cast<uint2*>(qr + v * E) = make_uint2(packed[0], packed[1]);
-            } else {
-                *reinterpret_cast<uint32_t*>(qr + v * E) = packed[0];
-            }
-        }
+        if (v < nvec) quant_vec_store<Tin>(regs[i], qrow, qr + v * E);
     }
 }
 
@@ -212,6 +291,18 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
     if (nvec <= 256 && rows >= 4 * (int64_t)num_sms && zero_n == 0 && ldx == K && ldq == K) {
         // many short rows (the MoE requant): a warp per row
         quant_rows_warp_kernel<Tin><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(x, rows, K, q, s);
+        return cudaGetLastError();
+    }
+    if (rows >= 2 * (int64_t)num_sms && nvec * 16 <= kQuantSmemRowMax) {
+        const int nt = nvec >= 128 ? 128 : 64;
+        const size_t smem = (size_t)nvec * 16;
+        auto kern = nt == 128 ? quant_rows_smem_kernel<Tin, 128> : quant_rows_smem_kernel<Tin, 64>;
+        if (smem > 48 * 1024) {
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+        kern<<<(unsigned)rows, nt, smem, stream>>>(x, K, ldx, q, ldq, s, zero_buf, zero_n);
         return cudaGetLastError();
     }
     int NT, cl;

@@ -120,12 +120,20 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 # ------------------------------------------------------------------ quant
 
 def quant_act(x: torch.Tensor, stream=None):
-    """Per-token int8 quant of bf16 x [M,K] -> (codes int8 [M,K], scales fp32 [M])."""
-    _need(x, torch.bfloat16, "x", 2)
+    """Per-token int8 quant of bf16 x [M,K] -> (codes int8 [M,K], scales fp32 [M]).
+
+    x may be a row-strided view (unit column stride, row stride = ldx)."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise TypeError("x must be a CUDA tensor")
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
     M, K = x.shape
+    ldx = x.stride(0) if M > 1 else K
+    if x.stride(1) != 1 or ldx < K:
+        raise ValueError("x rows must be contiguous (unit column stride, row stride >= K)")
     q = torch.empty((M, K), dtype=torch.int8, device=x.device)
     s = torch.empty(M, dtype=torch.float32, device=x.device)
-    _check(lib().w8a8_quant_act(_ptr(x), M, K, K, _ptr(q), _ptr(s), _stream(stream)), "w8a8_quant_act")
+    _check(lib().w8a8_quant_act(_ptr(x), M, K, ldx, _ptr(q), _ptr(s), _stream(stream)), "w8a8_quant_act")
     return q, s
 
 

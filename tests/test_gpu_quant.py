@@ -78,3 +78,46 @@ def test_quant_near_ties_take_the_exact_path(orc):
     qo, so = orc.quant_rows_f32(w)
     assert np.array_equal(q.cpu().numpy(), qo)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+@pytest.mark.parametrize("M,K", [(300, 512), (400, 17408), (296, 2064), (700, 1024), (300, 104448)])
+def test_quant_act_many_rows(orc, M, K):
+    """Row counts of a prefill batch: rows staged in shared memory (one and two
+    CTA widths), the warp-per-row kernel, and rows too long to stage."""
+    xb, _ = inputs.dense_linear(M * 3 + K, M, K, 16, with_weights=False)
+    _check_act(orc, xb)
+
+
+@pytest.mark.parametrize("N,K", [(300, 256), (320, 17408), (600, 1024)])
+def test_quant_rows_f32_many_rows(orc, N, K):
+    w = inputs.weights(np.random.default_rng(N + K), (N, K))
+    q, s = w8a8.quant_rows_f32(torch.from_numpy(w).cuda())
+    qo, so = orc.quant_rows_f32(w)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_quant_act_row_stride(orc):
+    """x is every other row block of a wider buffer (ldx > K), many rows."""
+    xb, _ = inputs.dense_linear(5, 320, 6144, 16, with_weights=False)
+    full = to_dev_bf16(xb)
+    view = full[:, 1024:1024 + 4096]
+    q, s = w8a8.quant_act(view)
+    qo, so = orc.quant_rows_bf16(np.ascontiguousarray(xb[:, 1024:1024 + 4096]))
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_quant_special_values_many_rows(orc):
+    """Special rows repeated past the row count that switches kernels."""
+    rows = np.zeros((6, 64), np.float32)
+    rows[1, 3] = -1e-40
+    rows[2] = np.array([127, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, 126.5] * 8, np.float32) / 16
+    rows[3] = -np.abs(np.linspace(0.1, 3, 64))
+    rows[4] = np.float32(3.0e38) * np.sign(np.sin(np.arange(64)))
+    rows[5, ::2] = -0.0
+    _check_act(orc, inputs.to_bf16_bits(np.tile(rows, (60, 1))))
+    q, s = w8a8.quant_rows_f32(torch.from_numpy(np.tile(rows, (60, 1))).cuda())
+    qo, so = orc.quant_rows_f32(np.tile(rows, (60, 1)))
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
