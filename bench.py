@@ -11,6 +11,7 @@ roofline fraction.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--quick]   (headline only, no extra workloads)
+    python bench.py --case NAME (one small workload for a profiler capture)
 
 Multi-GPU: the path has no exchange step; N ranks run independent replicas
 (weak scaling), timed on the device, max over ranks.
@@ -450,6 +451,68 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
     return out
 
 
+# --------------------------------------------------------------------------- profiling cases
+CASES = ("gemv_gateup_m8", "gemv_down_m8", "prefill_gateup_m512", "prefill_down_m512", "prefill_gateup_m4096",
+         "prefill_down_m4096", "quant_m4096_k17408", "quant_m4096_k5120", "moe_t1", "moe_t8", "moe_t512",
+         "moe_t4096", "hadamard_m1", "hadamard_m2048")
+
+
+def run_case(name, torch, dev, reps=4):
+    """One small named workload for an ncu capture: inputs drawn on the device
+    (seeded), the kernel of interest launched `reps` times, no timing."""
+    from moe_gemm_absmax_b200 import inputs, w8a8
+    w8a8.lib()
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+
+    def randn(*shape, std=1.0):
+        return torch.randn(*shape, generator=g, device=dev) * std
+
+    kind, _, rest = name.partition("_")
+    if kind in ("gemv", "prefill"):
+        which, m = rest.split("_")
+        d = inputs.GATE_UP if which == "gateup" else inputs.DOWN
+        M = int(m[1:])
+        qw, sw = w8a8.quant_rows_f32(randn(d["N"], d["K"], std=0.02))
+        qx, sx = w8a8.quant_act(randn(M, d["K"]).to(torch.bfloat16))
+        path = w8a8.PATH_GEMV if kind == "gemv" else w8a8.PATH_TCGEN05
+        y = torch.empty((M, d["N"]), dtype=torch.bfloat16, device=dev)
+        torch.cuda.empty_cache()      # only live buffers stay on the device during the capture
+        for _ in range(reps):
+            w8a8.gemm_q(qx, sx, qw, sw, path, y=y)
+    elif kind == "quant":
+        m, k = rest.split("_")
+        x = randn(int(m[1:]), int(k[1:])).to(torch.bfloat16)
+        for _ in range(reps):
+            w8a8.quant_act(x)
+    elif kind == "moe":
+        T = int(rest[1:])
+        E, H, I, k = inputs.MOE["E"], inputs.MOE["H"], inputs.MOE["I"], inputs.MOE["topk"]
+        q13, s13 = w8a8.quant_rows_f32(randn(E, 2 * I, H, std=0.02))
+        q2, s2 = w8a8.quant_rows_f32(randn(E, H, I, std=0.02))
+        x = randn(T, H).to(torch.bfloat16)
+        lg = randn(T, E).to(torch.bfloat16)
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.moe_workspace_size(T, E, H, I, k), dtype=torch.uint8, device=dev)
+        torch.cuda.empty_cache()
+        for _ in range(reps):
+            w8a8.moe_forward(x, lg, q13, s13, q2, s2, k, y=y, ws=ws)
+    elif kind == "hadamard":
+        M = int(rest[1:])
+        d = inputs.HADAMARD
+        qw, sw = w8a8.fwht128_quant(randn(d["N"], d["K"], std=0.02).to(torch.bfloat16))
+        x = randn(M, d["K"]).to(torch.bfloat16)
+        y = torch.empty((M, d["N"]), dtype=torch.bfloat16, device=dev)
+        torch.cuda.empty_cache()
+        for _ in range(reps):
+            q, s = w8a8.fwht128_quant(x)
+            w8a8.linear_g128(q, s, qw, sw, y=y)
+    else:
+        raise SystemExit(f"unknown case {name}; one of {', '.join(CASES)}")
+    torch.cuda.synchronize()
+    print(f"case {name}: ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -457,7 +520,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--quick", action="store_true")
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run one small named workload for a profiler capture and exit")
     args = ap.parse_args()
+    if args.case is not None:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        run_case(args.case, torch, dev)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -294,9 +294,18 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
         return cudaGetLastError();
     }
     if (rows >= 2 * (int64_t)num_sms && nvec * 16 <= kQuantSmemRowMax) {
-        const int nt = nvec >= 128 ? 128 : 64;
         const size_t smem = (size_t)nvec * 16;
-        auto kern = nt == 128 ? quant_rows_smem_kernel<Tin, 128> : quant_rows_smem_kernel<Tin, 64>;
+        int rows_per_sm = (int)((228 * 1024) / (smem + 1024));
+        rows_per_sm = rows_per_sm < 1 ? 1 : (rows_per_sm > 32 ? 32 : rows_per_sm);
+        // threads per CTA: fill the SM's 2048 threads so that the dependent ALU
+        // chains of the quantization overlap across warps -- with 16 or more
+        // rows resident 128 threads do (64 from 32 rows); with fewer, the
+        // largest power of two that keeps every row that fits resident
+        int nt = rows_per_sm >= 32 ? 64 : 128;
+        while (rows_per_sm < 16 && nt < 512 && rows_per_sm * nt * 2 <= 2048) nt *= 2;
+        auto kern = nt == 512 ? quant_rows_smem_kernel<Tin, 512>
+                  : nt == 256 ? quant_rows_smem_kernel<Tin, 256>
+                  : nt == 128 ? quant_rows_smem_kernel<Tin, 128> : quant_rows_smem_kernel<Tin, 64>;
         if (smem > 48 * 1024) {
             const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
