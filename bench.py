@@ -454,7 +454,7 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
 # --------------------------------------------------------------------------- profiling cases
 CASES = ("gemv_gateup_m8", "gemv_down_m8", "prefill_gateup_m512", "prefill_down_m512", "prefill_gateup_m4096",
          "prefill_down_m4096", "quant_m4096_k17408", "quant_m4096_k5120", "moe_t1", "moe_t8", "moe_t512",
-         "moe_t4096", "hadamard_m1", "hadamard_m2048")
+         "moe_t4096", "hadamard_m1", "hadamard_m200", "hadamard_m2048")
 
 
 def run_case(name, torch, dev, reps=4):

@@ -30,7 +30,6 @@ namespace w8a8 {
 
 constexpr int kTcBM = 128;
 constexpr int kTcBK = 128;          // int8 elements (= bytes) of K per stage: one swizzle atom
-constexpr int kTcThreads = 192;
 constexpr int kKernelIdGemmTc = 1;
 
 // Epilogues: dense bf16, raw int32, group-128 promotion, and the two grouped
@@ -110,7 +109,10 @@ struct TcSmem {
     static constexpr int kB = BN * kTcBK;                    // bytes per B stage
     static constexpr int kTiles = STAGES * (kA + kB);
     static constexpr int kBars = (2 * STAGES + 2 * 4 + 1) * 8;
-    static constexpr int kBytes = 1024 /*alignment slack*/ + kTiles + kBars + 16;
+    // epilogue scratch (group-128 column scales): 8 warps x 64 fp32
+    static constexpr int kEpiOff = kTiles + (kBars + 16 + 15) / 16 * 16;
+    static constexpr int kEpiBytes = 8 * 64 * 4;
+    static constexpr int kBytes = 1024 /*alignment slack*/ + kEpiOff + kEpiBytes;
 };
 
 // NEPI epilogue warps: 4 (one per TMEM lane quarter) or 8 (two per quarter,
@@ -122,12 +124,11 @@ template <int BN, int STAGES, int EPI, int NACC, bool GROUPED = false, int NEPI 
 __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
     gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
     static_assert(NEPI == 4 || NEPI == 8, "epilogue warps");
-    static_assert(NEPI == 4 || EPI != kEpiG128, "group-128 epilogue uses 4 warps");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(NACC >= 2 && NACC <= 4, "NACC");
     constexpr int kCols = NACC * BN;
     static_assert(kCols == 64 || kCols == 128 || kCols == 256 || kCols == 512, "TMEM columns: power of two");
-    static_assert(EPI != kEpiG128 || BN <= 128, "group-128 epilogue keeps BN fp32 sums per thread");
+    static_assert(EPI != kEpiG128 || BN * 4 / NEPI <= 128, "group-128 epilogue keeps its columns' fp32 sums");
     using SM = TcSmem<BN, STAGES>;
 
     extern __shared__ uint8_t smem_raw[];
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
     uint64_t* mma_done = tempty + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* epi_scratch = reinterpret_cast<float*>(smem + SM::kEpiOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -221,8 +223,11 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                 for (int kb = 0; kb < p.num_k_blocks; ++kb) {
                     const bool new_acc = (EPI == kEpiG128) || kb == 0;
                     if (new_acc) {
-                        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag,
-                                               (kKernelIdGemmTc << 16) | 3)) {
+                        // group-128: the epilogue refills each buffer with the
+                        // conversion bias and releases it once more at the start,
+                        // so its first use waits for phase 0 as well
+                        const uint32_t par = EPI == kEpiG128 ? acc_phase : (acc_phase ^ 1u);
+                        if (!mbar_wait_bounded(&tempty[acc], par, abort_flag, (kKernelIdGemmTc << 16) | 3)) {
                             ok = false;
                             break;
                         }
@@ -238,7 +243,7 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                     const uint32_t b0 = smem_u32(sB + stage * SM::kB);
 #pragma unroll
                     for (int kk = 0; kk < kTcBK / 32; ++kk) {
-                        const bool accumulate = kk > 0 || (EPI != kEpiG128 && kb > 0);
+                        const bool accumulate = EPI == kEpiG128 || kk > 0 || kb > 0;
                         tc_mma_i8(d_tmem, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
                                   accumulate ? 1u : 0u);
                     }
@@ -269,6 +274,17 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
+        if constexpr (EPI == kEpiG128) {
+            // every accumulator buffer starts from the conversion bias
+            constexpr int kStep = NEPI == 8 ? 64 : 32;
+            const uint32_t tq0 = tmem_base + ((uint32_t)(quarter * 32) << 16);
+            for (int b = 0; b < NACC; ++b)
+                for (int c = (NEPI == 8 ? 32 * chalf : 0); c < BN; c += kStep)
+                    tmem_st_32x32b_x32_fill(tq0 + (uint32_t)(b * BN + c), 0x4B400000u);
+            tc_wait_st();
+            tc_fence_before();
+            for (int b = 0; b < NACC; ++b) mbar_arrive(&tempty[b]);
+        }
         for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
             const TcTile ti = tc_tile<GROUPED, BN>(p, tile);
             const int nt = ti.n0 / BN;
@@ -276,34 +292,78 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
             const bool row_ok = row_in_tile < ti.valid;
             const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
             if constexpr (EPI == kEpiG128) {
+                // y[row, col] = sum over groups g ascending of
+                //   fma(float(p_g), sx[row, g] * sw[col, g], y)   (fp32), then * 1/128.
+                // Two columns per instruction (f32x2).  Each accumulator buffer
+                // starts from the bias 0x4B400000 (the bits of 1.5 * 2^23)
+                // instead of zero, so it ends holding the float bits of
+                // 1.5 * 2^23 + p_g exactly (|p_g| <= 127^2 * 128 < 2^22) and
+                // float(p_g) is one subtraction.  The 32 column scales of a chunk
+                // go through this warp's shared scratch, read back as 4-wide
+                // broadcasts.
+                constexpr int kStep = NEPI == 8 ? 64 : 32;   // column distance between this warp's chunks
+                constexpr int kChunks = BN / kStep;
+                const int c0 = NEPI == 8 ? 32 * chalf : 0;
                 const int G = p.num_k_blocks;
-                float y[BN];
+                const uint64_t magic2 = 0x4B4000004B400000ull;
+                float* wsc = epi_scratch + (warp - 2) * 64;
+                uint64_t y2[kChunks * 16];
 #pragma unroll
-                for (int j = 0; j < BN; ++j) y[j] = 0.0f;
+                for (int j = 0; j < kChunks * 16; ++j) y2[j] = 0ull;
+                float sx_next = row_ok ? bf16_bits_to_float(__ldg(p.gsx + (int64_t)row * G)) : 0.0f;
+                float sw_next[kChunks];
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    const int col = nt * BN + c0 + i * kStep + lane;
+                    sw_next[i] = col < p.N ? bf16_bits_to_float(__ldg(p.gsw + (int64_t)col * G)) : 0.0f;
+                }
                 for (int kb = 0; kb < G; ++kb) {
+                    const float sxg = sx_next;
+                    __syncwarp();   // the previous group's broadcast reads are done
+#pragma unroll
+                    for (int i = 0; i < kChunks; ++i) wsc[i * 32 + lane] = sw_next[i];
+                    __syncwarp();
+                    if (kb + 1 < G) {   // next group's scales, in flight during this group
+                        sx_next = row_ok ? bf16_bits_to_float(__ldg(p.gsx + (int64_t)row * G + kb + 1)) : 0.0f;
+#pragma unroll
+                        for (int i = 0; i < kChunks; ++i) {
+                            const int col = nt * BN + c0 + i * kStep + lane;
+                            sw_next[i] = col < p.N ? bf16_bits_to_float(__ldg(p.gsw + (int64_t)col * G + kb + 1)) : 0.0f;
+                        }
+                    }
                     if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const float sxg = row_ok ? bf16_bits_to_float(__ldg(p.gsx + (int64_t)row * G + kb)) : 0.0f;
+                    // chunk by chunk: into registers, the bias back into TMEM, the
+                    // promotion; the buffer goes back to the MMA after the last chunk
+                    const uint64_t sx2 = f2_pack(sxg, sxg);
 #pragma unroll
-                    for (int c = 0; c < BN; c += 32) {
+                    for (int i = 0; i < kChunks; ++i) {
+                        const uint32_t ta = tq + (uint32_t)(acc * BN + c0 + i * kStep);
                         uint32_t r[32];
-                        tmem_ld_32x32b_x32(tq + (uint32_t)(acc * BN + c), r);
-                        // lane i fetches the weight scale of column n0 + i; shuffles share it
-                        const int ncol = nt * BN + c + lane;
-                        const float swl =
-                            ncol < p.N ? bf16_bits_to_float(__ldg(p.gsw + (int64_t)ncol * G + kb)) : 0.0f;
+                        tmem_ld_32x32b_x32(ta, r);
                         tc_wait_ld();
+                        tmem_st_32x32b_x32_fill(ta, 0x4B400000u);
+                        if (i == kChunks - 1) {
+                            tc_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(&tempty[acc]);
+                        }
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float sc = __fmul_rn(sxg, __shfl_sync(0xffffffffu, swl, j));
-                            y[c + j] = __fmaf_rn(__int2float_rn((int)r[j]), sc, y[c + j]);
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 s4 = *reinterpret_cast<const float4*>(wsc + i * 32 + 4 * q);
+                            const uint64_t sc01 = f2_mul(sx2, f2_pack(s4.x, s4.y));
+                            const uint64_t sc23 = f2_mul(sx2, f2_pack(s4.z, s4.w));
+                            const uint64_t p01 =
+                                f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
+                            const uint64_t p23 =
+                                f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
+                            y2[i * 16 + 2 * q] = f2_fma(p01, sc01, y2[i * 16 + 2 * q]);
+                            y2[i * 16 + 2 * q + 1] = f2_fma(p23, sc23, y2[i * 16 + 2 * q + 1]);
                         }
                     }
-                    tc_fence_before();
-                    mbar_arrive(&tempty[acc]);
                     if (++acc == NACC) {
                         acc = 0;
                         acc_phase ^= 1u;
@@ -311,16 +371,22 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                 }
                 if (ok && row_ok) {
                     uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
+                    const uint64_t inv2 = f2_pack(0.0078125f, 0.0078125f);
 #pragma unroll
-                    for (int v = 0; v < BN / 8; ++v) {
-                        const int n0 = nt * BN + v * 8;
-                        if (n0 < p.N) {
-                            uint32_t pk[4];
+                    for (int i = 0; i < kChunks; ++i) {
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                pk[j] = pack_bf16x2(__fmul_rn(y[v * 8 + 2 * j], 0.0078125f),
-                                                    __fmul_rn(y[v * 8 + 2 * j + 1], 0.0078125f));
-                            *reinterpret_cast<uint4*>(yrow + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        for (int v = 0; v < 4; ++v) {
+                            const int n0 = nt * BN + c0 + i * kStep + v * 8;
+                            if (n0 < p.N) {
+                                uint32_t pk[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    float a, b;
+                                    f2_unpack(f2_mul(y2[i * 16 + v * 4 + j], inv2), a, b);
+                                    pk[j] = pack_bf16x2(a, b);
+                                }
+                                *reinterpret_cast<uint4*>(yrow + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            }
                         }
                     }
                 }

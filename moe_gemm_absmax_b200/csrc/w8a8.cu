@@ -82,10 +82,10 @@ bool make_tmap_i8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
 }
 
 // ----------------------------------------------------------------- tcgen05 GEMM
-template <int BN, int STAGES, int EPI, int NACC>
+template <int BN, int STAGES, int EPI, int NACC, int NEPI = 4>
 int launch_tc(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     using SM = TcSmem<BN, STAGES>;
-    auto kern = gemm_i8_tc_kernel<BN, STAGES, EPI, NACC>;
+    auto kern = gemm_i8_tc_kernel<BN, STAGES, EPI, NACC, false, NEPI>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
     static bool attr_done[kMaxDevices] = {false};
@@ -103,7 +103,7 @@ int launch_tc(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
     const int tiles = p.num_m_tiles * p.num_n_tiles;
     const int grid = tiles < device_sms(dev) ? tiles : device_sms(dev);
-    kern<<<grid, kTcThreads, SM::kBytes, st>>>(ta, tb, p);
+    kern<<<grid, tc_threads<NEPI>(), SM::kBytes, st>>>(ta, tb, p);
     return last_launch_status();
 }
 
@@ -771,7 +771,7 @@ int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, con
     p.gsx = sx;
     p.gsw = sw;
     p.out = y;
-    return launch_tc<128, 6, kEpiG128, 4>(qx, qw, p, st);
+    return launch_tc<128, 6, kEpiG128, 4, 8>(qx, qw, p, st);
 }
 
 // ----------------------------------------------------------------- diagnostics
