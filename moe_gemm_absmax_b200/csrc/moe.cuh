@@ -50,15 +50,18 @@ struct MoePlan {
     int32_t* offsets;    // [E + 1]
     int32_t* active;     // [E] touched experts, ascending
     int32_t* n_active;   // [1]
-    int32_t* tile_off;   // [E + 1] prefix sum of ceil(counts / 128): grouped-GEMM row tiles
+    int32_t* tile_off;   // [E + 1] prefix sum of ceil(counts / tile_rows): grouped-GEMM row tiles
     int32_t* rank;       // [T * topk] rank of (token, slot) inside its expert
     int32_t* done;       // [1] finished CTAs
+    int tile_rows;       // rows per tile of the grouped GEMMs that follow
 };
 
 template <int EPL>
 __global__ void __launch_bounds__(256) moe_route_plan_kernel(const uint16_t* __restrict__ logits, int64_t T, int E,
                                                              int topk, int32_t* __restrict__ ids,
                                                              float* __restrict__ wts, MoePlan p) {
+    // the scatter that follows may start its launch now; it waits for this grid
+    asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
     if (t < T) {
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(256) moe_route_plan_kernel(const uint16_t* __r
     __threadfence();
     const int e = threadIdx.x;
     const int c = e < E ? __ldcg(p.counts + e) : 0;
-    const int mt = (c + 127) / 128;
+    const int mt = (c + p.tile_rows - 1) / p.tile_rows;
     auto block_excl_scan = [&](int v) {   // exclusive scan over the 256 threads; returns (excl, total)
         int incl = v;
 #pragma unroll
@@ -196,6 +199,10 @@ __global__ void __launch_bounds__(1024) moe_quant_scatter_kernel(const uint16_t*
                                                                  int8_t* __restrict__ dbg_qx,
                                                                  float* __restrict__ dbg_sx) {
     const int64_t t = blockIdx.x;
+    // the plan comes from the kernel just before; the next kernel may launch
+    // once every CTA is past this wait (so the plan is complete by then)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     // sorted rows of this token's slots (and their metadata)
     __shared__ int srow[kMoeMaxTopk];
     if (threadIdx.x < topk) {
@@ -347,6 +354,7 @@ __global__ void __launch_bounds__(kGemvThreads) moe_gemm_kernel(MoeGemmArgs m) {
 // already-combined [T, H] buffer.
 __global__ void moe_finalize_kernel(const float* __restrict__ contrib, uint16_t* __restrict__ y, int64_t T, int H,
                                     int topk) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // contrib comes from the kernel just before
     const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (i >= T * H) return;
     const int64_t t = i / H, n = i % H;

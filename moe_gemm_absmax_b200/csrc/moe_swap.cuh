@@ -1,0 +1,324 @@
+// Routed-expert GEMMs (a8 + a9 and a10 + a11) on the 5th-generation tensor
+// cores, swap-AB -- "Online INT8 W8A8 ...", Changes (MoE pipeline: fused
+// gated-SiLU via interleaved w13, per-token int8 quant before gemm2, gemm2
+// with weighted scatter/combine).
+//
+// With a few to a few dozen rows per expert, the expert's weights are the
+// 128-row A operand of tcgen05.mma.kind::i8 and its rows' codes the narrow B
+// operand (N = BN = 16, 32 or 64 rows of one expert):
+//   D[n, m] = sum_k W_e[n, k] X[r_m, k]     (TMEM: lane = weight row n, column = row m)
+// so each MMA reads a 128 x 32 weight slice at full rate and the kernel runs
+// at the speed TMA streams the touched experts' weights out of HBM.
+//
+// Work unit: (token block, 128-row weight group) with the whole K; token
+// blocks are BN consecutive expert-sorted rows of one expert (the plan's
+// tile_off counts them per expert).  Units are dealt round-robin to a
+// persistent grid; unit u = block * ngroups + group, so the groups of one
+// block run side by side and the blocks of one expert reuse its weights
+// through L2.
+//
+// gemm1 epilogue (GATED): v = (float(acc) * sx[r]) * s13[e, n]; rows n = 2i
+// (gate) and 2i + 1 (up) sit in neighbouring lanes; a[r, i] = SiLU(g) * u,
+// fp32.  gemm2 epilogue: y2 = (float(acc) * sa[r]) * s2[e, n]; w_r * y2
+// stored at (token, slot) for the slot-order combine.
+//
+// Launched with programmatic dependent launch: the routing plan is complete
+// when a kernel of this chain starts (each kernel of the chain lets its
+// successor start only after its own wait on its predecessor, and the plan
+// comes two or more kernels back), so the producer reads the plan and starts
+// the weight tiles of its first stages before it waits for the codes of the
+// kernel just before.
+//
+// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+// warps 2..5 epilogue (TMEM lane quarters).  All waits are bounded.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace w8a8 {
+
+constexpr int kMsBM = 128;          // weight rows per group (MMA M)
+constexpr int kMsBK = 128;          // bytes of K per stage
+constexpr int kMsThreads = 192;
+constexpr int kKernelIdMoeSwap = 5;
+
+template <int BN>
+struct MsSmem {
+    static constexpr int kStages = BN <= 32 ? 10 : 8;
+    static constexpr int kW = kMsBM * kMsBK;        // 16 KB
+    static constexpr int kX = BN * kMsBK;           // 2 / 4 / 8 KB
+    static constexpr int kStage = kW + kX;          // multiple of 1024
+    static constexpr int kTiles = kStages * kStage;
+    static constexpr int kBars = (2 * kStages + 4 + 1) * 8;
+    // the plan (tile_off, offsets, counts: 3 x 257 ints) and, per epilogue
+    // buffer, the token block's row data (scale, destination, weight)
+    static constexpr int kPlanOff = kTiles + kBars + 16;
+    static constexpr int kPlanInts = 3 * 260;
+    static constexpr int kRowOff = kPlanOff + kPlanInts * 4;
+    static constexpr int kRowBytes = 2 * 3 * 64 * 4;
+    static constexpr int kBytes = 1024 + kRowOff + kRowBytes;
+};
+
+struct MoeSwapArgs {
+    const float* sw;          // [E, rows] weight-row scales
+    const float* sx;          // [R] scales of the sorted rows (gemm1: x codes, gemm2: a codes)
+    const int32_t* counts;    // [E]
+    const int32_t* offsets;   // [E + 1]
+    const int32_t* tile_off;  // [E + 1] prefix of ceil(counts / BN)
+    int E, rows, K;           // rows: 2I (gemm1) or H (gemm2)
+    int ngroups, nkb;         // rows / 128, K / 128
+    // gemm1
+    float* a_out;             // [R, I] fp32 gated intermediate
+    // gemm2
+    const int32_t* row_tok;   // [R]
+    const int32_t* row_slot;  // [R]
+    const float* row_w;       // [R]
+    float* contrib;           // [T * topk, H] w * y2 at (token, slot)
+    int topk;
+};
+
+// Token block b (in tile_off numbering) -> expert, first sorted row, rows;
+// the plan's arrays in shared memory (sp: tile_off [E + 1], offsets, counts).
+struct MsBlock {
+    int e, row0, valid;
+};
+
+__device__ __forceinline__ MsBlock ms_block(const int* sp, int E, int b, int BN) {
+    const int* tile_off = sp;
+    const int* offsets = sp + 260;
+    const int* counts = sp + 520;
+    int lo = 0, hi = E;   // largest e with tile_off[e] <= b (experts without rows own no block)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tile_off[mid] <= b) lo = mid;
+        else hi = mid;
+    }
+    MsBlock k;
+    k.e = lo;
+    const int lb = b - tile_off[lo];
+    k.row0 = offsets[lo] + lb * BN;
+    k.valid = min(BN, counts[lo] - lb * BN);
+    return k;
+}
+
+__device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN, bool GATED>
+__global__ void __launch_bounds__(kMsThreads, 1)
+    moe_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, MoeSwapArgs a) {
+    static_assert(BN == 16 || BN == 32 || BN == 64, "BN");
+    using SM = MsSmem<BN>;
+    constexpr int STAGES = SM::kStages;
+    constexpr int kCols = 2 * BN >= 32 ? 2 * BN : 32;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kTiles);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // The plan is complete (see above); the codes of the kernel just before may not be.
+    int* sp = reinterpret_cast<int*>(smem + SM::kPlanOff);
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
+        sp[i] = __ldg(a.tile_off + i);
+        sp[260 + i] = __ldg(a.offsets + i);
+        sp[520 + i] = i < a.E ? __ldg(a.counts + i) : 0;
+    }
+    __syncthreads();
+    const int nunits = sp[a.E] * a.ngroups;
+    const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int64_t my_stages = (int64_t)my_units * a.nkb;
+    const int pre = my_stages < STAGES ? (int)my_stages : STAGES;   // stages armed before the wait
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmW);
+        prefetch_tensormap(&tmX);
+        for (int i = 0; i < pre; ++i) {   // unit blockIdx.x + (i / nkb) * gridDim.x, k block i % nkb
+            const int u = blockIdx.x + (i / a.nkb) * gridDim.x;
+            const int b = u / a.ngroups, g = u - b * a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            mbar_arrive_expect_tx(&full[i], (uint32_t)SM::kStage);
+            tma_load_2d(smem + i * SM::kStage, &tmW, &full[i], (i % a.nkb) * kMsBK, k.e * a.rows + g * kMsBM);
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, last_phase = 0;
+            int64_t i = 0;   // stage count of this CTA
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const int b = u / a.ngroups, g = u - b * a.ngroups;
+                const MsBlock k = ms_block(sp, a.E, b, BN);
+                const int wrow = k.e * a.rows + g * kMsBM;
+                for (int kb = 0; kb < a.nkb; ++kb, ++i) {
+                    if (i >= pre) {
+                        if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, (kKernelIdMoeSwap << 16) | 1)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[stage], (uint32_t)SM::kStage);
+                        tma_load_2d(smem + stage * SM::kStage, &tmW, &full[stage], kb * kMsBK, wrow);
+                    }
+                    tma_load_2d(smem + stage * SM::kStage + SM::kW, &tmX, &full[stage], kb * kMsBK, k.row0);
+                    issued |= 1u << stage;
+                    last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: every copy this thread started lands before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait_bounded(&full[s], (last_phase >> s) & 1u, nullptr, (kKernelIdMoeSwap << 16) | 2,
+                                          100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(kMsBM, BN);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, (kKernelIdMoeSwap << 16) | 3)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < a.nkb; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, (kKernelIdMoeSwap << 16) | 4)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t w0 = smem_u32(smem + stage * SM::kStage);
+                    const uint32_t x0 = w0 + SM::kW;
+#pragma unroll
+                    for (int kk = 0; kk < kMsBK / 32; ++kk)
+                        tc_mma_i8(d_tmem, smem_desc_k_sw128(w0 + kk * 32), smem_desc_k_sw128(x0 + kk * 32), idesc,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            tc_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0u, nullptr, (kKernelIdMoeSwap << 16) | 5, 100000000ull);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int et = threadIdx.x - 64;   // 0 .. 127
+        float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff);   // [2][3][64]
+        int acc = 0, buf = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+            const int b = u / a.ngroups, g = u - b * a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            // the block's row data, one row per thread, before the accumulator is ready
+            float* rs = s_row + buf * 3 * 64;
+            if (et < BN) {
+                const int r = k.row0 + et;
+                const bool have = et < k.valid;
+                rs[et] = have ? __ldg(a.sx + r) : 0.0f;
+                if constexpr (!GATED) {
+                    rs[64 + et] = __int_as_float(have ? __ldg(a.row_tok + r) * a.topk + __ldg(a.row_slot + r) : 0);
+                    rs[128 + et] = have ? __ldg(a.row_w + r) : 0.0f;
+                }
+            }
+            ms_epi_sync();   // also: every warp is done with this buffer's use two units ago
+            buf ^= 1;
+            if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) break;
+            tc_fence_after();
+            int v[BN];
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll
+            for (int c = 0; c < BN; c += 16) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(taddr + (uint32_t)c, r);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[c + j] = (int)r[j];
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+            const int n = g * kMsBM + quarter * 32 + lane;   // weight row of expert e
+            const float swn = __ldg(a.sw + (int64_t)k.e * a.rows + n);
+            if constexpr (GATED) {
+                const int I = a.rows >> 1;
+                float* arow = a.a_out + (int64_t)k.row0 * I + (n >> 1);
+#pragma unroll
+                for (int m = 0; m < BN; ++m) {
+                    const float val = __fmul_rn(__fmul_rn(__int2float_rn(v[m]), rs[m]), swn);
+                    const float up = __shfl_xor_sync(0xffffffffu, val, 1);   // row n + 1 (odd lane)
+                    if (m < k.valid && !(lane & 1)) arow[(int64_t)m * I] = __fmul_rn(silu_proj(val), up);
+                }
+            } else {
+                const int H = a.rows;
+#pragma unroll
+                for (int m = 0; m < BN; ++m) {
+                    if (m < k.valid) {
+                        const float y2 = __fmul_rn(__fmul_rn(__int2float_rn(v[m]), rs[m]), swn);
+                        a.contrib[(int64_t)__float_as_int(rs[64 + m]) * H + n] = __fmul_rn(rs[128 + m], y2);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kCols);
+    }
+}
+
+}  // namespace w8a8

@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(NT) quant_rows_smem_kernel(const Tin* __restri
     constexpr int E = VT::kElems;
     extern __shared__ __align__(16) uint4 row_s[];
     asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // x may come from the kernel just before
     const int64_t row = blockIdx.x;
     const int nvec = (int)(K / E);
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
     // let a kernel launched after this one with programmatic serialization
     // start its independent prologue now (it still waits for our results)
     asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // x may come from the kernel just before
     // optional side job: clear a small int buffer that a later kernel on the
     // same stream expects to find zero (split-K arrival counters)
     for (int i = blockIdx.x * NT + threadIdx.x; i < zero_n; i += gridDim.x * NT) zero_buf[i] = 0;
@@ -244,6 +246,8 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
     using VT = VecTraits<Tin>;
     constexpr int E = VT::kElems;
     constexpr int kMaxV = 8;
+    asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // x may come from the kernel just before
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -285,13 +289,22 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
 //              more SMs pull the row from HBM.
 template <typename Tin>
 cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* s,
-                              cudaStream_t stream, int num_sms, int* zero_buf = nullptr, int zero_n = 0) {
+                              cudaStream_t stream, int num_sms, int* zero_buf = nullptr, int zero_n = 0,
+                              bool pdl = false) {
+    cudaLaunchAttribute pdl_attr[1];
+    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
     constexpr int E = VecTraits<Tin>::kElems;
     const int64_t nvec = K / E;
     if (nvec <= 256 && rows >= 4 * (int64_t)num_sms && zero_n == 0 && ldx == K && ldq == K) {
         // many short rows (the MoE requant): a warp per row
-        quant_rows_warp_kernel<Tin><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(x, rows, K, q, s);
-        return cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((rows + 7) / 8), 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = stream;
+        cfg.attrs = pdl_attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        return cudaLaunchKernelEx(&cfg, quant_rows_warp_kernel<Tin>, x, rows, K, q, s);
     }
     if (rows >= 2 * (int64_t)num_sms && nvec * 16 <= kQuantSmemRowMax) {
         const size_t smem = (size_t)nvec * 16;
@@ -311,8 +324,14 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
             if (e != cudaSuccess) return e;
         }
         if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
-        kern<<<(unsigned)rows, nt, smem, stream>>>(x, K, ldx, q, ldq, s, zero_buf, zero_n);
-        return cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)rows, 1, 1);
+        cfg.blockDim = dim3((unsigned)nt, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cfg.attrs = pdl_attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        return cudaLaunchKernelEx(&cfg, kern, x, K, ldx, q, ldq, s, zero_buf, zero_n);
     }
     int NT, cl;
     if (rows >= 2 * (int64_t)num_sms && nvec <= 1024 * 6) {
@@ -336,13 +355,18 @@ cudaError_t launch_quant_rows(const Tin* x, int64_t rows, int64_t K, int64_t ldx
     cfg.blockDim = dim3((unsigned)NT, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (cl > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)cl;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) attr[na++] = pdl_attr[0];
     cfg.attrs = attr;
-    cfg.numAttrs = cl > 1 ? 1 : 0;
+    cfg.numAttrs = na;
 #define W8A8_QUANT_LAUNCH(nt, mv) \
     return cudaLaunchKernelEx(&cfg, quant_rows_kernel<Tin, nt, mv>, x, K, ldx, q, ldq, s, vpc, cl, zero_buf, zero_n)
     switch (NT) {

@@ -16,6 +16,7 @@
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
 #include "moe.cuh"
+#include "moe_swap.cuh"
 #include "quant.cuh"
 #include "w8a8.h"
 
@@ -379,6 +380,9 @@ struct MoeWs {
 constexpr size_t kMoeExactCombineBytes = (size_t)64 << 20;
 inline bool moe_exact_combine(int64_t R, int H) { return (size_t)R * H * 4 <= kMoeExactCombineBytes; }
 
+// Token blocks of the swap path: at most one partial block per touched expert.
+inline int64_t moe_max_blocks(int64_t R, int E, int bn) { return R / bn + (R < E ? R : E) + 1; }
+
 MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     MoeWs w;
     const int64_t R = T * topk;
@@ -391,7 +395,7 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     };
     w.ids = reinterpret_cast<int32_t*>(take((size_t)R * 4));
     w.wts = reinterpret_cast<float*>(take((size_t)R * 4));
-    // counts and the CTA counter are adjacent: one memset clears both
+    // counts and the plan's CTA counter are adjacent: one memset clears both
     w.counts = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
     w.done = w.counts + E;
     w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
@@ -439,6 +443,48 @@ int launch_tc_grouped(const int8_t* A, int64_t rowsA, const int8_t* B, int E, Tc
     p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
     kern<<<device_sms(dev), tc_threads<NEPI>(), SM::kBytes, st>>>(ta, tb, p);
     return last_launch_status();
+}
+
+// Swap-AB expert GEMM over token blocks of BN rows: W = an expert stack
+// viewed as [E * rows, K], X = the sorted codes [R, K].
+template <int BN, bool GATED>
+int launch_moe_swap(const int8_t* W, const int8_t* X, int64_t R, MoeSwapArgs a, int64_t nb_max, cudaStream_t st) {
+    using SM = MsSmem<BN>;
+    auto kern = moe_swap_kernel<BN, GATED>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    static bool attr_done[kMaxDevices] = {false};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    CUtensorMap tw, tx;
+    if (!make_tmap_i8(&tw, W, (uint64_t)a.E * a.rows, (uint64_t)a.K, kMsBM)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tx, X, (uint64_t)R, (uint64_t)a.K, BN)) return W8A8_ERR_CUDA;
+    const int64_t units = nb_max * a.ngroups;
+    const int sms = device_sms(dev);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units < sms ? units : sms), 1, 1);
+    cfg.blockDim = dim3(kMsThreads, 1, 1);
+    cfg.dynamicSmemBytes = SM::kBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    pdl_config(cfg, at, true);
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tw, tx, a));
+}
+
+// A plain kernel launch on the MoE chain, with programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+int launch_chained(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    pdl_config(cfg, at, true);
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, args...));
 }
 
 template <int WN, int WK, int TG, bool GATED>
@@ -611,6 +657,28 @@ int w8a8_gemm_s32(const int8_t* qx, const int8_t* qw, int32_t* acc, int64_t M, i
 }
 
 
+}  // extern "C"
+
+namespace {
+// Optional parity outputs of the MoE forward (a debug struct given by the caller).
+int moe_debug_copies(const MoeWs& w, const w8a8_moe_debug* dbg, int64_t R, int E, int I, cudaStream_t st) {
+    if (!dbg) return W8A8_OK;
+    if (dbg->topk_ids && cudaMemcpyAsync(dbg->topk_ids, w.ids, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
+        return W8A8_ERR_CUDA;
+    if (dbg->topk_w && cudaMemcpyAsync(dbg->topk_w, w.wts, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
+        return W8A8_ERR_CUDA;
+    if (dbg->counts && cudaMemcpyAsync(dbg->counts, w.counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, st))
+        return W8A8_ERR_CUDA;
+    if (dbg->qa || dbg->sa) {
+        moe_debug_gather_kernel<<<(unsigned)R, 128, 0, st>>>(w.qa, w.sa, w.row_of, R, I, dbg->qa, dbg->sa);
+        return last_launch_status();
+    }
+    return W8A8_OK;
+}
+}  // namespace
+
+extern "C" {
+
 size_t w8a8_moe_workspace_size(int64_t T, int E, int H, int I, int topk) {
     if (T <= 0 || E <= 0 || H <= 0 || I <= 0 || topk <= 0) return 0;
     return moe_carve(nullptr, T, E, H, I, topk).bytes;
@@ -633,18 +701,64 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     const int64_t R = T * topk;
     int rc;
 
+    const bool exact_combine = moe_exact_combine(R, H);
+    // up to a few dozen rows per expert: swap-AB expert GEMMs with the requant
+    // and the combine fused in (weights streamed once per token block)
+    const int64_t avg_rows = (R + E - 1) / E;
+    const bool swap = exact_combine && H % 128 == 0 && I % 128 == 0 && I <= 2048 && avg_rows <= 64;
+    const int swap_bn = avg_rows <= 12 ? 16 : (avg_rows <= 24 ? 32 : 64);
     if (cudaMemsetAsync(w.counts, 0, (size_t)(E + 1) * 4, st) != cudaSuccess) return W8A8_ERR_CUDA;
-    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.rank, w.done};
+    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.rank, w.done, swap ? swap_bn : 128};
     moe_route_plan_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts, plan);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
-    const bool exact_combine = moe_exact_combine(R, H);
     MoeRows rows = {w.ids, w.wts, w.rank, w.offsets, w.row_of, w.row_tok, w.row_slot, w.row_w};
-    moe_quant_scatter_kernel<<<(unsigned)T, (unsigned)((H / 8 + 31) / 32 * 32), 0, st>>>(
-        x, H, topk, rows, w.xq, w.sxr, exact_combine ? nullptr : w.out, dbg ? dbg->qx : nullptr,
-        dbg ? dbg->sx : nullptr);
-    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+    rc = launch_chained(moe_quant_scatter_kernel, (unsigned)T, (unsigned)((H / 8 + 31) / 32 * 32), st, x, H, topk,
+                        rows, w.xq, w.sxr, exact_combine ? (float*)nullptr : w.out,
+                        dbg ? dbg->qx : (int8_t*)nullptr, dbg ? dbg->sx : (float*)nullptr);
+    if (rc != W8A8_OK) return rc;
 
+    if (swap) {
+        const int64_t nb_max = moe_max_blocks(R, E, swap_bn);
+        MoeSwapArgs a1 = {};
+        a1.sw = s13;
+        a1.sx = w.sxr;
+        a1.counts = w.counts;
+        a1.offsets = w.offsets;
+        a1.tile_off = w.tile_off;
+        a1.E = E;
+        a1.rows = 2 * I;
+        a1.K = H;
+        a1.ngroups = (2 * I) / 128;
+        a1.nkb = H / 128;
+        a1.a_out = w.a;
+        MoeSwapArgs a2 = a1;
+        a2.sw = s2;
+        a2.sx = w.sa;
+        a2.rows = H;
+        a2.K = I;
+        a2.ngroups = H / 128;
+        a2.nkb = I / 128;
+        a2.row_tok = w.row_tok;
+        a2.row_slot = w.row_slot;
+        a2.row_w = w.row_w;
+        a2.contrib = w.out;
+        a2.topk = topk;
+        rc = swap_bn == 16 ? launch_moe_swap<16, true>(w13, w.xq, R, a1, nb_max, st)
+           : swap_bn == 32 ? launch_moe_swap<32, true>(w13, w.xq, R, a1, nb_max, st)
+                           : launch_moe_swap<64, true>(w13, w.xq, R, a1, nb_max, st);
+        if (rc != W8A8_OK) return rc;
+        if (launch_quant_rows<float>(w.a, R, I, I, w.qa, I, w.sa, st, current_sms(), nullptr, 0, true) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        rc = swap_bn == 16 ? launch_moe_swap<16, false>(w2, w.qa, R, a2, nb_max, st)
+           : swap_bn == 32 ? launch_moe_swap<32, false>(w2, w.qa, R, a2, nb_max, st)
+                           : launch_moe_swap<64, false>(w2, w.qa, R, a2, nb_max, st);
+        if (rc != W8A8_OK) return rc;
+        rc = launch_chained(moe_finalize_kernel, (unsigned)((T * H / 4 + 255) / 256), 256u, st, (const float*)w.out,
+                            y, T, H, topk);
+        if (rc != W8A8_OK) return rc;
+        return moe_debug_copies(w, dbg, R, E, I, st);
+    }
     const int max_active = (int)(R < E ? R : E);
     const bool wide = R > (int64_t)E * 8;   // more than 8 rows per expert on average
     // many rows per expert: grouped tcgen05 GEMMs over 128-row tiles of each expert's rows
@@ -726,19 +840,7 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     moe_finalize_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, st>>>(w.out, y, T, H, exact_combine ? topk : 1);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
-    if (dbg) {
-        if (dbg->topk_ids && cudaMemcpyAsync(dbg->topk_ids, w.ids, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-        if (dbg->topk_w && cudaMemcpyAsync(dbg->topk_w, w.wts, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-        if (dbg->counts && cudaMemcpyAsync(dbg->counts, w.counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-        if (dbg->qa || dbg->sa) {
-            moe_debug_gather_kernel<<<(unsigned)R, 128, 0, st>>>(w.qa, w.sa, w.row_of, R, I, dbg->qa, dbg->sa);
-            if ((rc = last_launch_status()) != W8A8_OK) return rc;
-        }
-    }
-    return W8A8_OK;
+    return moe_debug_copies(w, dbg, R, E, I, st);
 }
 
 // ----------------------------------------------------------------- FWHT128

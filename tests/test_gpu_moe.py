@@ -71,9 +71,14 @@ def _small(seed, T, E, H, I, skew=None):
 @pytest.mark.parametrize("T,E,H,I,k,skew", [(5, 8, 256, 64, 2, None), (37, 8, 256, 64, 2, None),
                                              (40, 16, 512, 128, 2, 3), (1, 4, 128, 64, 4, None),
                                              (9, 256, 2048, 512, 8, None),
-                                             # grouped tcgen05 path: >= 16 rows per expert
-                                             (64, 4, 256, 128, 2, None), (300, 4, 256, 128, 2, 1),
-                                             (520, 8, 512, 256, 3, 5)])
+                                             # swap-AB expert GEMMs: token blocks of 16 / 32 / 64 rows,
+                                             # several blocks per expert under skew, I up to 2048,
+                                             # a single 128-column group (H = 128)
+                                             (48, 8, 256, 128, 4, None), (64, 4, 256, 128, 2, None),
+                                             (100, 8, 256, 128, 4, None), (200, 8, 256, 128, 2, 2),
+                                             (12, 4, 256, 2048, 2, None), (7, 8, 128, 128, 2, None),
+                                             # 128-row tile path: more rows per expert
+                                             (300, 4, 256, 128, 2, 1), (520, 8, 512, 256, 3, 5)])
 def test_moe_small_configs(orc, T, E, H, I, k, skew):
     xb, lb, w13, w2 = _small(T * 31 + E, T, E, H, I, skew)
     gw = _quant_experts_gpu(w13, w2)
