@@ -56,6 +56,111 @@ struct MoePlan {
     int tile_rows;       // rows per tile of the grouped GEMMs that follow
 };
 
+// Total order of bf16 logits as unsigned 16-bit keys (NaN taken as -inf,
+// -0 as +0, so equal values get equal keys).
+__device__ __forceinline__ uint32_t logit_key16(uint16_t b) {
+    if ((b & 0x7fffu) > 0x7f80u) b = 0xff80u;   // NaN -> -inf
+    if (b == 0x8000u) b = 0u;                   // -0 -> +0
+    return (b & 0x8000u) ? (~(uint32_t)b & 0xffffu) : ((uint32_t)b | 0x8000u);
+}
+
+// a5 for one token, by one warp: lane l holds experts l, l + 32, ...
+// (E <= 32 * EPL).  p = softmax(l) in fp32 with the project exponential and
+// the denominator summed in expert-index order (staged in ex_s, this warp's
+// 32 * EPL floats of shared memory, one lane folds them); top-k by logit,
+// ties to the lower expert index: each expert's key is (ordered logit << 16)
+// | (0xffff - e), so the largest key is the largest logit with the smallest
+// index, and one warp max-reduction picks each slot.  Lane j < topk returns
+// slot j's expert and its weight p_j / sum over the k of p (slot order).
+template <int EPL>
+__device__ __forceinline__ void route_token(const uint16_t* __restrict__ lrow, int E, int topk, float* ex_s,
+                                            int& id_j, float& w_j) {
+    const int lane = threadIdx.x & 31;
+    float l[EPL];
+    uint32_t key[EPL];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            const uint16_t b = __ldg(lrow + e);
+            l[i] = bf16_bits_to_float(b);
+            if (isnan(l[i])) l[i] = -INFINITY;   // out of domain; keeps the selection well defined
+            key[i] = (logit_key16(b) << 16) | (0xffffu - (uint32_t)e);
+        } else {
+            l[i] = -INFINITY;
+            key[i] = 0u;
+        }
+        mx = fmaxf(mx, l[i]);
+    }
+    mx = warp_max(mx);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        ex_s[lane + 32 * i] = e < E ? exp_proj(__fsub_rn(l[i], mx)) : 0.0f;
+    }
+    __syncwarp();
+    float sum = 0.0f;
+    if (lane == 0) {
+#pragma unroll 8
+        for (int e = 0; e < E; ++e) sum = __fadd_rn(sum, ex_s[e]);
+    }
+    sum = __shfl_sync(0xffffffffu, sum, 0);
+    id_j = 0;
+    for (int j = 0; j < topk; ++j) {
+        uint32_t kl = key[0];
+#pragma unroll
+        for (int i = 1; i < EPL; ++i) kl = max(kl, key[i]);
+        const uint32_t km = __reduce_max_sync(0xffffffffu, kl);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (key[i] == km) key[i] = 0u;   // taken (keys are distinct: the index is in them)
+        if (lane == j) id_j = (int)(0xffffu - (km & 0xffffu));
+    }
+    const float p_j = lane < topk ? __fdiv_rn(ex_s[id_j], sum) : 0.0f;
+    float ssel = 0.0f;
+    for (int j = 0; j < topk; ++j) ssel = __fadd_rn(ssel, __shfl_sync(0xffffffffu, p_j, j));
+    w_j = lane < topk ? __fdiv_rn(p_j, ssel) : 0.0f;
+}
+
+// Exclusive scan of one int per thread over the whole CTA (at most 16
+// warps); returns (exclusive prefix, total).  Every thread of the CTA calls it.
+__device__ __forceinline__ int2 block_excl_scan(int v, int* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    __syncthreads();
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+        if (w < warp) before += warp_tot[w];
+        total += warp_tot[w];
+    }
+    return make_int2(incl - v + before, total);
+}
+
+// a6: thread e (< E; one expert per thread, E <= blockDim.x) holds count c;
+// writes offsets, tile offsets in tiles of tile_rows rows and the list of
+// touched experts.  Returns the expert's offset.
+__device__ __forceinline__ int moe_plan_write(int c, int E, const MoePlan& p, int* warp_tot) {
+    const int e = threadIdx.x;
+    const int2 off = block_excl_scan(c, warp_tot);
+    if (e < E) p.offsets[e] = off.x;
+    if (e == 0) p.offsets[E] = off.y;
+    const int2 toff = block_excl_scan((c + p.tile_rows - 1) / p.tile_rows, warp_tot);
+    if (e < E) p.tile_off[e] = toff.x;
+    if (e == 0) p.tile_off[E] = toff.y;
+    const int2 act = block_excl_scan(c > 0 ? 1 : 0, warp_tot);
+    if (e < E && c > 0) p.active[act.x] = e;
+    if (e == 0) p.n_active[0] = act.y;
+    return off.x;
+}
+
 template <int EPL>
 __global__ void __launch_bounds__(256) moe_route_plan_kernel(const uint16_t* __restrict__ logits, int64_t T, int E,
                                                              int topk, int32_t* __restrict__ ids,
@@ -64,81 +169,21 @@ __global__ void __launch_bounds__(256) moe_route_plan_kernel(const uint16_t* __r
     asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    __shared__ float ex_s[8][32 * EPL];
     if (t < T) {
-        float l[EPL], ex[EPL];
-        bool taken[EPL];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int e = lane + 32 * i;
-            l[i] = e < E ? bf16_bits_to_float(logits[t * E + e]) : -INFINITY;
-            if (isnan(l[i])) l[i] = -INFINITY;   // out of domain; keeps the selection well defined
-            taken[i] = e >= E;
-            mx = fmaxf(mx, l[i]);
-        }
-        mx = warp_max(mx);
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int e = lane + 32 * i;
-            ex[i] = e < E ? exp_proj(__fsub_rn(l[i], mx)) : 0.0f;
-        }
-        // softmax denominator summed in expert-index order, as a serial loop
-        // would: stage the exponentials, one lane folds them, then broadcast
-        __shared__ float ex_s[8][32 * EPL];
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) ex_s[warp][lane + 32 * i] = ex[i];
-        __syncwarp();
-        float sum = 0.0f;
-        if (lane == 0)
-            for (int e = 0; e < E; ++e) sum = __fadd_rn(sum, ex_s[warp][e]);
-        sum = __shfl_sync(0xffffffffu, sum, 0);
-
-        float psel_j = 0.0f;   // lane j keeps the probability of slot j
-        int id_j = 0;
-        for (int j = 0; j < topk; ++j) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            float bex = 0.0f;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int e = lane + 32 * i;
-                if (!taken[i] && (l[i] > bv || (l[i] == bv && e < bi))) {
-                    bv = l[i];
-                    bi = e;
-                    bex = ex[i];
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                const float oex = __shfl_xor_sync(0xffffffffu, bex, o);
-                if (ov > bv || (ov == bv && oi < bi)) {
-                    bv = ov;
-                    bi = oi;
-                    bex = oex;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (lane + 32 * i == bi) taken[i] = true;
-            if (lane == j) {
-                id_j = bi;
-                psel_j = __fdiv_rn(bex, sum);
-            }
-        }
-        float ssel = 0.0f;
-        for (int j = 0; j < topk; ++j) ssel = __fadd_rn(ssel, __shfl_sync(0xffffffffu, psel_j, j));
+        int id_j;
+        float w_j;
+        route_token<EPL>(logits + t * E, E, topk, ex_s[warp], id_j, w_j);
         if (lane < topk) {
             ids[t * topk + lane] = id_j;
-            wts[t * topk + lane] = __fdiv_rn(psel_j, ssel);
+            wts[t * topk + lane] = w_j;
             p.rank[t * topk + lane] = atomicAdd(p.counts + id_j, 1);
         }
     }
 
     // ---- the last CTA scans the histogram (E <= 256: one expert per thread)
     __shared__ int last;
-    __shared__ int warp_tot[8];
+    __shared__ int warp_tot[16];
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) last = (atomicAdd(p.done, 1) == (int)gridDim.x - 1);
@@ -146,35 +191,7 @@ __global__ void __launch_bounds__(256) moe_route_plan_kernel(const uint16_t* __r
     if (!last) return;
     __threadfence();
     const int e = threadIdx.x;
-    const int c = e < E ? __ldcg(p.counts + e) : 0;
-    const int mt = (c + p.tile_rows - 1) / p.tile_rows;
-    auto block_excl_scan = [&](int v) {   // exclusive scan over the 256 threads; returns (excl, total)
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += u;
-        }
-        __syncthreads();
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        int before = 0, total = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            if (w < warp) before += warp_tot[w];
-            total += warp_tot[w];
-        }
-        return make_int2(incl - v + before, total);
-    };
-    const int2 off = block_excl_scan(c);
-    if (e < E) p.offsets[e] = off.x;
-    if (e == 0) p.offsets[E] = off.y;
-    const int2 toff = block_excl_scan(mt);
-    if (e < E) p.tile_off[e] = toff.x;
-    if (e == 0) p.tile_off[E] = toff.y;
-    const int2 act = block_excl_scan(c > 0 ? 1 : 0);
-    if (e < E && c > 0) p.active[act.x] = e;
-    if (e == 0) p.n_active[0] = act.y;
+    moe_plan_write(e < E ? __ldcg(p.counts + e) : 0, E, p, warp_tot);
 }
 
 // ---------------------------------------------------------------------------
@@ -258,6 +275,85 @@ __global__ void __launch_bounds__(1024) moe_quant_scatter_kernel(const uint16_t*
         float4* o = reinterpret_cast<float4*>(clear_rows + t * H) + 2 * v;
         o[0] = make_float4(0.f, 0.f, 0.f, 0.f);
         o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a5 + a6 + a7 for a few tokens (T <= 16) in one CTA of 16 warps, warp t
+// handling token t: routing, ranks from a shared-memory histogram (so the
+// plan needs no cleared global counters), the plan scan, then the token's
+// int8 codes written once per routed slot into the expert-sorted rows.
+constexpr int kMoeFrontMaxT = 16;
+
+template <int EPL>
+__global__ void __launch_bounds__(512) moe_front_small_kernel(const uint16_t* __restrict__ x,
+                                                              const uint16_t* __restrict__ logits, int T, int E,
+                                                              int H, int topk, int32_t* __restrict__ ids,
+                                                              float* __restrict__ wts, MoePlan p, MoeRows rows,
+                                                              int8_t* __restrict__ xq, float* __restrict__ sxr,
+                                                              int8_t* __restrict__ dbg_qx,
+                                                              float* __restrict__ dbg_sx) {
+    // the GEMM that follows reads nothing of ours before its own wait
+    asm volatile("griddepcontrol.launch_dependents;");
+    __shared__ int s_cnt[256];
+    __shared__ int s_off[256];
+    __shared__ int s_rows[kMoeFrontMaxT][kMoeMaxTopk];
+    __shared__ float ex_s[kMoeFrontMaxT][32 * EPL];
+    __shared__ int warp_tot[16];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    int id_j = 0, rank_j = 0;
+    float w_j = 0.0f;
+    if (warp < T) {
+        route_token<EPL>(logits + (int64_t)warp * E, E, topk, ex_s[warp], id_j, w_j);
+        if (lane < topk) {
+            rank_j = atomicAdd(&s_cnt[id_j], 1);
+            ids[warp * topk + lane] = id_j;
+            wts[warp * topk + lane] = w_j;
+            p.rank[warp * topk + lane] = rank_j;
+        }
+    }
+    __syncthreads();
+    const int e = threadIdx.x;
+    const int c = e < E ? s_cnt[e] : 0;
+    if (e < E) p.counts[e] = c;
+    const int off = moe_plan_write(c, E, p, warp_tot);
+    if (e < E) s_off[e] = off;
+    __syncthreads();
+    if (warp >= T) return;
+    if (lane < topk) {
+        const int r = s_off[id_j] + rank_j;
+        s_rows[warp][lane] = r;
+        rows.row_of[warp * topk + lane] = r;
+        rows.row_tok[r] = warp;
+        rows.row_slot[r] = lane;
+        rows.row_w[r] = w_j;
+    }
+    __syncwarp();
+    // a7: the token's codes (two passes over its row; the second hits L1)
+    using VT = VecTraits<uint16_t>;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)warp * H);
+    const int nvec = H / 8;
+    VT::Acc acc = VT::acc_init();
+    for (int v = lane; v < nvec; v += 32) VT::acc(acc, __ldg(xr + v));
+    float amax;
+    if (!VT::acc_final(acc, amax)) {   // NaN among this lane's values
+        amax = 0.0f;
+        for (int v = lane; v < nvec; v += 32) amax = fmaxf(amax, vec_absmax<uint16_t>(__ldg(xr + v)));
+    }
+    const QuantRow q(warp_max(amax));
+    if (lane < topk) sxr[s_rows[warp][lane]] = q.s;
+    if (dbg_sx && lane == 0) dbg_sx[warp] = q.s;
+    for (int v = lane; v < nvec; v += 32) {
+        float f[8];
+        VT::unpack(__ldg(xr + v), f);
+        uint32_t pk[2];
+        quant_codes<2>(f, q, pk);
+        const uint2 codes = make_uint2(pk[0], pk[1]);
+        for (int j = 0; j < topk; ++j)
+            *reinterpret_cast<uint2*>(xq + (int64_t)s_rows[warp][j] * H + v * 8) = codes;
+        if (dbg_qx) *reinterpret_cast<uint2*>(dbg_qx + (int64_t)warp * H + v * 8) = codes;
     }
 }
 

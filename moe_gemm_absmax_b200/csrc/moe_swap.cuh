@@ -76,6 +76,7 @@ struct MoeSwapArgs {
     const float* row_w;       // [R]
     float* contrib;           // [T * topk, H] w * y2 at (token, slot)
     int topk;
+    int early_plan;           // the plan comes two or more kernels back: read it before the wait
 };
 
 // Token block b (in tile_off numbering) -> expert, first sorted row, rows;
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kMsThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // The plan is complete (see above); the codes of the kernel just before may not be.
+    if (!a.early_plan) asm volatile("griddepcontrol.wait;" ::: "memory");
     int* sp = reinterpret_cast<int*>(smem + SM::kPlanOff);
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
         sp[i] = __ldg(a.tile_off + i);

@@ -707,16 +707,23 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     const int64_t avg_rows = (R + E - 1) / E;
     const bool swap = exact_combine && H % 128 == 0 && I % 128 == 0 && I <= 2048 && avg_rows <= 64;
     const int swap_bn = avg_rows <= 12 ? 16 : (avg_rows <= 24 ? 32 : 64);
-    if (cudaMemsetAsync(w.counts, 0, (size_t)(E + 1) * 4, st) != cudaSuccess) return W8A8_ERR_CUDA;
     MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.rank, w.done, swap ? swap_bn : 128};
-    moe_route_plan_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts, plan);
-    if ((rc = last_launch_status()) != W8A8_OK) return rc;
-
     MoeRows rows = {w.ids, w.wts, w.rank, w.offsets, w.row_of, w.row_tok, w.row_slot, w.row_w};
-    rc = launch_chained(moe_quant_scatter_kernel, (unsigned)T, (unsigned)((H / 8 + 31) / 32 * 32), st, x, H, topk,
-                        rows, w.xq, w.sxr, exact_combine ? (float*)nullptr : w.out,
-                        dbg ? dbg->qx : (int8_t*)nullptr, dbg ? dbg->sx : (float*)nullptr);
-    if (rc != W8A8_OK) return rc;
+    const bool front_small = T <= kMoeFrontMaxT && exact_combine;
+    if (front_small) {
+        // routing, plan and x codes in one CTA
+        moe_front_small_kernel<8><<<1, 512, 0, st>>>(x, logits, (int)T, E, H, topk, w.ids, w.wts, plan, rows, w.xq,
+                                                     w.sxr, dbg ? dbg->qx : nullptr, dbg ? dbg->sx : nullptr);
+        if ((rc = last_launch_status()) != W8A8_OK) return rc;
+    } else {
+        if (cudaMemsetAsync(w.counts, 0, (size_t)(E + 1) * 4, st) != cudaSuccess) return W8A8_ERR_CUDA;
+        moe_route_plan_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts, plan);
+        if ((rc = last_launch_status()) != W8A8_OK) return rc;
+        rc = launch_chained(moe_quant_scatter_kernel, (unsigned)T, (unsigned)((H / 8 + 31) / 32 * 32), st, x, H,
+                            topk, rows, w.xq, w.sxr, exact_combine ? (float*)nullptr : w.out,
+                            dbg ? dbg->qx : (int8_t*)nullptr, dbg ? dbg->sx : (float*)nullptr);
+        if (rc != W8A8_OK) return rc;
+    }
 
     if (swap) {
         const int64_t nb_max = moe_max_blocks(R, E, swap_bn);
@@ -732,7 +739,9 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
         a1.ngroups = (2 * I) / 128;
         a1.nkb = H / 128;
         a1.a_out = w.a;
+        a1.early_plan = front_small ? 0 : 1;   // after the front kernel the plan is one kernel back
         MoeSwapArgs a2 = a1;
+        a2.early_plan = 1;
         a2.sw = s2;
         a2.sx = w.sa;
         a2.rows = H;
