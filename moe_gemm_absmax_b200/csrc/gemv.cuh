@@ -65,7 +65,7 @@ template <int WN, int WK, int TG, class RowMap, int U = kGemvUnroll, bool PF = f
 __device__ __forceinline__ bool gemv_core(const GemvShape& a, int (&acc)[TG][4], int& block_out, int kseg = 0,
                                           int nkseg = 1, int ctr = 0) {
     static_assert(WN * WK == kGemvThreads / 32, "8 warps");
-    __shared__ int red[WK > 1 ? WK - 1 : 1][WN][TG][32][4];
+    __shared__ __align__(16) int red[WK > 1 ? WK - 1 : 1][WN][TG][32][4];   // read and written as int4
     __shared__ int is_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
