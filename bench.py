@@ -155,6 +155,26 @@ def time_events(torch, fn, iters, flush=None):
     return float(np.mean(ts)), float(np.median(ts))
 
 
+def graph_events(torch, fn, iters, flush=None):
+    """Mean device time in ms of one replay of a CUDA graph that holds fn()
+    (captured after warm-up on a side stream), CUDA events around each replay."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    t, _ = time_events(torch, g.replay, iters, flush=flush)
+    del g
+    return t
+
+
 def local_gpu_index(torch):
     """nvidia-smi index of this process's GPU (first entry of CUDA_VISIBLE_DEVICES if set)."""
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
@@ -332,6 +352,17 @@ def run_ours(args, rank, world, torch, dev):
                 "timing": "kernel alone, CUDA events per launch, L2 evicted by a read between launches",
                 "peak_source": peaks["source"] + " (burst copy)"}
 
+    # ---- the down-proj GEMV alone, and the whole step replayed from a CUDA graph
+    qxd, sxd = w8a8.quant_act(xs["down"])
+    Nd, Kd = W["down"][0].shape
+    y_d = torch.empty((M, Nd), dtype=torch.bfloat16, device=dev)
+    dfn = lambda: w8a8.gemm_q(qxd, sxd, W["down"][0], W["down"][1], w8a8.PATH_GEMV, y=y_d)
+    for _ in range(3):
+        dfn()
+    d_ms, _ = time_events(torch, dfn, 20, flush=flush)
+    d_bytes = Nd * Kd + 4 * Nd + M * Kd + 4 * M + 2 * M * Nd
+    graph_ms = graph_events(torch, step, 20)
+
     # ---- end to end through the C ABI with host buffers: pinned x in, y out, each step
     hx = {n: xs[n].cpu().pin_memory() for n in order}
     hy = {n: torch.empty(ys[n].shape, dtype=torch.bfloat16).pin_memory() for n in order}
@@ -371,6 +402,13 @@ def run_ours(args, rank, world, torch, dev):
             "e2e": {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": 4 * args.steps, "extra": extra}
+    line["decode_detail"] = {
+        "down_gemv_alone": {"kernel": "gemv_dense_kernel<4,2,1,8> (down K=17408 -> N=5120, M=8)", "ms": d_ms,
+                            "gbs": d_bytes / (d_ms * 1e-3) / 1e9, "frac": d_bytes / (d_ms * 1e-3) / 1e9 / hbm,
+                            "algorithmic_bytes": d_bytes},
+        "gate_up_gemv_alone_ms": k_ms,
+        "step_graph_replay": {"ms_per_step": graph_ms, "value": weight_bytes / (graph_ms * 1e-3) / 1e9,
+                              "unit": "GB/s", "note": "the same step captured once in a CUDA graph, replayed"}}
     return line
 
 
@@ -399,6 +437,18 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
                              "unit": "TOPS", "frac": ops / (t_gemm * 1e-3) / 1e12 / int8_peak,
                              "peak_source": "2 x measured bf16 burst (dense int8 : bf16 = 2 : 1)"}}
             del x, y, ws, qx, sx
+    # ---- per-token activation quant alone (a1) at the prefill shape
+    for K in (5120, 17408):
+        xq_in = bf16_dev(torch, inputs.dense_linear(5, 4096, K, 16, with_weights=False)[0], dev)
+        qfn = lambda: w8a8.quant_act(xq_in)
+        for _ in range(3):
+            qfn()
+        tq, _ = time_events(torch, qfn, 10, flush=flush)
+        qb = 4096 * K * 3 + 4096 * 4
+        out[f"act_quant_M4096_K{K}"] = {"ms": tq, "gbs": qb / (tq * 1e-3) / 1e9,
+                                        "roofline": {"bound": "hbm", "frac": qb / (tq * 1e-3) / 1e9 / hbm,
+                                                     "bytes": qb, "peak": hbm, "unit": "GB/s"}}
+        del xq_in
     # ---- routed MoE layer
     w13, w2 = inputs.moe_weights(0)
     q13, s13 = quantize_on_gpu(torch, w8a8, w13, dev)
@@ -415,10 +465,12 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         for _ in range(3):
             fn()
         t, _ = time_events(torch, fn, 10, flush=flush)
+        tg = graph_events(torch, fn, 10, flush=flush)
         _, dbg = w8a8.moe_forward(x, lg, q13, s13, q2, s2, 8, debug=True)
         touched = int((dbg["counts"] > 0).sum().item())
         byts = touched * per_expert + 2 * T * H * 2 + 2 * T * E
         out[f"moe_T{T}"] = {"ms": t, "tokens_per_s": T / (t * 1e-3), "touched_experts": touched,
+                            "graph_replay_ms": tg, "graph_replay_tokens_per_s": T / (tg * 1e-3),
                             "roofline": {"bound": "hbm", "achieved": byts / (t * 1e-3) / 1e9, "peak": hbm,
                                          "unit": "GB/s", "frac": byts / (t * 1e-3) / 1e9 / hbm,
                                          "bytes": byts}}
