@@ -348,7 +348,7 @@ def run_ours(args, rank, world, torch, dev):
     achieved = k_bytes / (k_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": recorded_traffic(), "algorithmic_bytes": k_bytes,
-                "kernel": "gemv_dense_kernel<4,2,1,8> (gate_up K=5120 -> N=34816, M=8)",
+                "kernel": "gemv_dense_kernel<4,2,1,4,4> (gate_up K=5120 -> N=34816, M=8)",
                 "timing": "kernel alone, CUDA events per launch, L2 evicted by a read between launches",
                 "peak_source": peaks["source"] + " (burst copy)"}
 
@@ -403,7 +403,7 @@ def run_ours(args, rank, world, torch, dev):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": 4 * args.steps, "extra": extra}
     line["decode_detail"] = {
-        "down_gemv_alone": {"kernel": "gemv_dense_kernel<4,2,1,8> (down K=17408 -> N=5120, M=8)", "ms": d_ms,
+        "down_gemv_alone": {"kernel": "gemv_dense_kernel<4,2,1,4,4> (down K=17408 -> N=5120, M=8)", "ms": d_ms,
                             "gbs": d_bytes / (d_ms * 1e-3) / 1e9, "frac": d_bytes / (d_ms * 1e-3) / 1e9 / hbm,
                             "algorithmic_bytes": d_bytes},
         "gate_up_gemv_alone_ms": k_ms,

@@ -99,6 +99,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// Programmatic dependent launch: a kernel launched to overlap the one before
+// it reads that kernel's results only after `griddepcontrol.wait`, and with
+// ordinary loads (__ldca / ld.global.ca where the SM's warps share the data,
+// __ldcg / ld.global.cg otherwise) or TMA: the compiler treats non-coherent
+// loads (__ldg, ld.global.nc) as invariant and may hoist them above the wait.
+// __ldg is kept for weights and for data written before the previous kernel
+// started.
+
 // ---------------------------------------------------------------------------
 // TMA (tiled, no multicast)
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {

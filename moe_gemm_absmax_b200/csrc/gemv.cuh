@@ -125,7 +125,7 @@ __device__ __forceinline__ bool gemv_core(const GemvShape& a, int (&acc)[TG][4],
                     const int tok = tg * 8 + g;
                     uint4 xb = make_uint4(0, 0, 0, 0);
                     if (tok < a.tokens && c + u < c1 && k < a.K)
-                        xb = __ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)tok * a.K + k));
+                        xb = __ldca(reinterpret_cast<const uint4*>(a.x + (int64_t)tok * a.K + k));   // L1: shared by the SM's warps
                     const uint32_t A1[4] = {wa[u].x, wb[u].x, wa[u].y, wb[u].y};
                     const uint32_t B1[2] = {xb.x, xb.y};
                     const uint32_t A2[4] = {wa[u].z, wb[u].z, wa[u].w, wb[u].w};
@@ -218,8 +218,11 @@ struct GemvEpiDense {
     int s32;           // 1: raw int32
 };
 
-template <int WN, int WK, int TG, int U>
-__global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(GemvShape a, GemvEpiDense e) {
+// MINB: resident CTAs per SM the register budget is sized for (4: 64
+// registers a thread, 32 warps an SM) -- the decode weight stream needs many
+// warps per SM with a few loads each, more than few warps with many loads.
+template <int WN, int WK, int TG, int U, int MINB = 1>
+__global__ void __launch_bounds__(kGemvThreads, MINB) gemv_dense_kernel(GemvShape a, GemvEpiDense e) {
     int acc[TG][4];
     int block;
     if (!gemv_core<WN, WK, TG, RowMapDense, U>(a, acc, block, blockIdx.y, gridDim.y, blockIdx.x)) return;
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(GemvShape a, G
                 if (e.s32) {
                     reinterpret_cast<int32_t*>(e.out)[(int64_t)m * e.N + n] = acc[tg][j];
                 } else {
-                    const float v = __fmul_rn(__fmul_rn(__int2float_rn(acc[tg][j]), __ldg(e.sx + m)), __ldg(e.sw + n));
+                    const float v = __fmul_rn(__fmul_rn(__int2float_rn(acc[tg][j]), __ldcg(e.sx + m)), __ldg(e.sw + n));
                     reinterpret_cast<uint16_t*>(e.out)[(int64_t)m * e.N + n] = float_to_bf16_bits(v);
                 }
             }

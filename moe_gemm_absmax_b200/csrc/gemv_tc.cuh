@@ -98,7 +98,7 @@ __device__ __forceinline__ void gc_store_row(const GemvTc& a, int n, const int (
             if (a.s32) {
                 reinterpret_cast<int32_t*>(a.out)[(int64_t)m * a.N + n] = v[m];
             } else {
-                const float r = __fmul_rn(__fmul_rn(__int2float_rn(v[m]), __ldg(a.sx + m)), swn);
+                const float r = __fmul_rn(__fmul_rn(__int2float_rn(v[m]), __ldcg(a.sx + m)), swn);
                 reinterpret_cast<uint16_t*>(a.out)[(int64_t)m * a.N + n] = float_to_bf16_bits(r);
             }
         }

@@ -224,12 +224,12 @@ __global__ void __launch_bounds__(1024) moe_quant_scatter_kernel(const uint16_t*
     __shared__ int srow[kMoeMaxTopk];
     if (threadIdx.x < topk) {
         const int64_t i = t * topk + threadIdx.x;
-        const int r = __ldg(rows.offsets + __ldg(rows.ids + i)) + __ldg(rows.rank + i);
+        const int r = __ldcg(rows.offsets + __ldcg(rows.ids + i)) + __ldcg(rows.rank + i);
         srow[threadIdx.x] = r;
         rows.row_of[i] = r;
         rows.row_tok[r] = (int)t;
         rows.row_slot[r] = threadIdx.x;
-        rows.row_w[r] = __ldg(rows.wts + i);
+        rows.row_w[r] = __ldcg(rows.wts + i);
     }
     const int v = threadIdx.x;          // vector index, 8 bf16
     const bool active = v < H / 8;

@@ -148,9 +148,9 @@ __global__ void __launch_bounds__(kMsThreads, 1)
     if (!a.early_plan) asm volatile("griddepcontrol.wait;" ::: "memory");
     int* sp = reinterpret_cast<int*>(smem + SM::kPlanOff);
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
-        sp[i] = __ldg(a.tile_off + i);
-        sp[260 + i] = __ldg(a.offsets + i);
-        sp[520 + i] = i < a.E ? __ldg(a.counts + i) : 0;
+        sp[i] = __ldcg(a.tile_off + i);
+        sp[260 + i] = __ldcg(a.offsets + i);
+        sp[520 + i] = i < a.E ? __ldcg(a.counts + i) : 0;
     }
     __syncthreads();
     const int nunits = sp[a.E] * a.ngroups;
@@ -265,10 +265,10 @@ __global__ void __launch_bounds__(kMsThreads, 1)
             if (et < BN) {
                 const int r = k.row0 + et;
                 const bool have = et < k.valid;
-                rs[et] = have ? __ldg(a.sx + r) : 0.0f;
+                rs[et] = have ? __ldcg(a.sx + r) : 0.0f;
                 if constexpr (!GATED) {
-                    rs[64 + et] = __int_as_float(have ? __ldg(a.row_tok + r) * a.topk + __ldg(a.row_slot + r) : 0);
-                    rs[128 + et] = have ? __ldg(a.row_w + r) : 0.0f;
+                    rs[64 + et] = __int_as_float(have ? __ldcg(a.row_tok + r) * a.topk + __ldcg(a.row_slot + r) : 0);
+                    rs[128 + et] = have ? __ldcg(a.row_w + r) : 0.0f;
                 }
             }
             ms_epi_sync();   // also: every warp is done with this buffer's use two units ago

@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
     for (int i = 0; i < MAXV; ++i) {
         const int64_t v = v0 + threadIdx.x + (int64_t)i * NT;
         if (v < v1) {
-            regs[i] = __ldg(xr + v);
+            regs[i] = __ldcg(xr + v);
             VT::acc(acc, regs[i]);
         }
     }

@@ -176,10 +176,11 @@ int run_tc(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw,
 
 // ----------------------------------------------------------------- GEMV
 // Decode GEMV.  M <= 8: the register-streaming mma.sync kernel
-// (gemv_dense_kernel): 4 row blocks x 2 K-halves per CTA, 8 chunks of
-// weight loads in flight per thread, and the K range split over `nkseg`
-// CTAs when the rows alone give too few CTAs (measured fastest for both
-// decode shapes).  9 <= M <= 32: the swap-AB tcgen05 kernel (gemv_tc_kernel),
+// (gemv_dense_kernel): 4 row blocks x 2 K-halves per CTA, 4 chunks of
+// weight loads in flight per thread, 64 registers so that 4 CTAs (32 warps)
+// stay resident per SM, and the K range split over `nkseg` CTAs until the
+// CTAs fill about 70% of those slots (measured fastest for both decode
+// shapes: more splits cost more in partial sums than they gain).  9 <= M <= 32: the swap-AB tcgen05 kernel (gemv_tc_kernel),
 // whose token columns grow for free.  Plans are fixed per shape
 // (independent of the device) so that workspace sizes are too.
 struct GemvPlan {
@@ -194,7 +195,7 @@ struct GemvPlan {
     int counters;
 };
 
-constexpr int kGemvWN = 4, kGemvWK = 2;
+constexpr int kGemvWN = 4, kGemvWK = 2, kGemvUnrollDecode = 4, kGemvMinBlocks = 4;
 constexpr int kGemvGrid = 148;
 constexpr int kGemvMaxM = 32;
 
@@ -207,7 +208,9 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
         g.ctas_x = (int)((blocks + kGemvWN - 1) / kGemvWN);
         const int64_t nchunks = (K + 63) / 64;
         int s = 1;
-        while (s < 8 && (int64_t)g.ctas_x * s < 160 && nchunks / (kGemvWK * s * 2) >= 8) s *= 2;
+        while (s < 16 && (int64_t)g.ctas_x * (s + 1) * 10 <= (int64_t)kGemvGrid * kGemvMinBlocks * 7 &&
+               nchunks / (kGemvWK * (s + 1)) >= 8)
+            ++s;
         g.nkseg = s;
         g.part_bytes = s > 1 ? align_up((size_t)s * blocks * g.tg * 32 * 16, 256) : 0;
         g.counters = s > 1 ? g.ctas_x : 0;
@@ -279,7 +282,7 @@ int launch_gemv_reg(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     pdl_config(cfg, at, after_quant);
-    return cuda_status(cudaLaunchKernelEx(&cfg, gemv_dense_kernel<kGemvWN, kGemvWK, TG, U>, a, e));
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemv_dense_kernel<kGemvWN, kGemvWK, TG, U, kGemvMinBlocks>, a, e));
 }
 
 // Runs the GEMV; `scratch` holds the partials and the counters (zero on entry).
@@ -302,7 +305,7 @@ int run_gemv(const int8_t* qx, const float* sx, const int8_t* qw, const float* s
         e.M = (int)M;
         e.N = (int)N;
         e.s32 = s32 ? 1 : 0;
-        return launch_gemv_reg<1, 8>(a, e, g, after_quant, st);
+        return launch_gemv_reg<1, kGemvUnrollDecode>(a, e, g, after_quant, st);
     }
     GemvTc a;
     a.sx = sx;
