@@ -77,17 +77,29 @@ __global__ void __launch_bounds__(256) fwht128_quant_kernel(const uint16_t* __re
 
 constexpr int kG128MaxGroups = 64;
 
-// One CTA per 16 weight rows; 8 warps split the K groups; tokens <= 8.
+// One CTA per 16 weight rows; 8 warps split the K groups; tokens <= 8.  The
+// scales of the CTA's rows and tokens are staged in shared memory first, so
+// that the serial per-group promotion of warp 0 reads no global memory.
 __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict__ qx,
                                                         const uint16_t* __restrict__ sx,
                                                         const int8_t* __restrict__ qw,
                                                         const uint16_t* __restrict__ sw, uint16_t* __restrict__ y,
                                                         int M, int N, int K) {
     __shared__ int4 pg[kG128MaxGroups][32];
+    __shared__ float s_sw[16][kG128MaxGroups];   // [row in CTA][group]
+    __shared__ float s_sx[8][kG128MaxGroups];    // [token][group]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t = lane & 3;
     const int G = K / 128;
     const int block = blockIdx.x;
+    for (int i = threadIdx.x; i < 16 * G; i += blockDim.x) {
+        const int r = i / G, grp = i - r * G, n = block * 16 + r;
+        s_sw[r][grp] = n < N ? bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp)) : 0.0f;
+    }
+    for (int i = threadIdx.x; i < 8 * G; i += blockDim.x) {
+        const int m = i / G, grp = i - m * G;
+        s_sx[m][grp] = m < M ? bf16_bits_to_float(__ldg(sx + (int64_t)m * G + grp)) : 0.0f;
+    }
     const int8_t* w0 = qw + (int64_t)(block * 16 + g8) * K + 16 * t;
     const int8_t* w1 = w0 + 8 * (int64_t)K;
     const bool tok_ok = g8 < M;
@@ -122,12 +134,8 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = 2 * t + (j & 1);
-            const int n = block * 16 + g8 + 8 * (j >> 1);
-            if (m < M) {
-                const float sc = __fmul_rn(bf16_bits_to_float(__ldg(sx + (int64_t)m * G + grp)),
-                                           bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp)));
-                yv[j] = __fmaf_rn(__int2float_rn(pv[j]), sc, yv[j]);
-            }
+            const int r = g8 + 8 * (j >> 1);
+            if (m < M) yv[j] = __fmaf_rn(__int2float_rn(pv[j]), __fmul_rn(s_sx[m][grp], s_sw[r][grp]), yv[j]);
         }
     }
 #pragma unroll

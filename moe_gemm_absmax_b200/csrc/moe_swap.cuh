@@ -257,19 +257,35 @@ __global__ void __launch_bounds__(kMsThreads, 1)
         float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff);   // [2][3][64]
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
+        // row data of a token block, one row per thread (et < BN): loaded one
+        // unit ahead so that its latency hides behind the current unit
+        float nx_sx = 0.0f, nx_w = 0.0f;
+        int nx_dst = 0;
+        auto fetch = [&](int u) {
+            const int b = u / a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            if (et < k.valid) {
+                const int r = k.row0 + et;
+                nx_sx = __ldcg(a.sx + r);
+                if constexpr (!GATED) {
+                    nx_dst = __ldcg(a.row_tok + r) * a.topk + __ldcg(a.row_slot + r);
+                    nx_w = __ldcg(a.row_w + r);
+                }
+            }
+        };
+        if (et < BN && (int)blockIdx.x < nunits) fetch(blockIdx.x);
         for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const int b = u / a.ngroups, g = u - b * a.ngroups;
             const MsBlock k = ms_block(sp, a.E, b, BN);
-            // the block's row data, one row per thread, before the accumulator is ready
             float* rs = s_row + buf * 3 * 64;
             if (et < BN) {
-                const int r = k.row0 + et;
                 const bool have = et < k.valid;
-                rs[et] = have ? __ldcg(a.sx + r) : 0.0f;
+                rs[et] = have ? nx_sx : 0.0f;
                 if constexpr (!GATED) {
-                    rs[64 + et] = __int_as_float(have ? __ldcg(a.row_tok + r) * a.topk + __ldcg(a.row_slot + r) : 0);
-                    rs[128 + et] = have ? __ldcg(a.row_w + r) : 0.0f;
+                    rs[64 + et] = __int_as_float(have ? nx_dst : 0);
+                    rs[128 + et] = have ? nx_w : 0.0f;
                 }
+                if (u + (int)gridDim.x < nunits) fetch(u + gridDim.x);
             }
             ms_epi_sync();   // also: every warp is done with this buffer's use two units ago
             buf ^= 1;

@@ -76,6 +76,7 @@ def lib():
             L.oracle_moe_histogram.argtypes = [vp, i64, i32, vp]
             L.oracle_moe_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32,
                                              vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.oracle_mlp_forward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
             L.oracle_fwht128.argtypes = [vp]
             L.oracle_fwht128_quant.argtypes = [vp, i64, i64, vp, vp, vp]
             L.oracle_gemm_g128.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
@@ -241,6 +242,25 @@ def moe_forward(x_bits, logits_bits, w13, s13, w2, s2, topk: int, tokens=None):
                              _p(out["ids"]), _p(out["wts"]), _p(out["qx"]), _p(out["sx"]),
                              _p(out["qa"]), _p(out["sa"]))
     out["tokens"] = toks
+    return out
+
+
+def mlp_forward(x_bits, w13, s13, w2, s2):
+    """Dense gated MLP block (x -> gate_up + SiLU*up -> requant -> down) for
+    all tokens.  w13 int8 [2I, H], s13 [2I], w2 int8 [H, I], s2 [H].
+    Returns a dict with y (bf16 bits), y32, qx, sx, qa, sa."""
+    x = _c(x_bits, np.uint16)
+    w13, w2 = _c(w13, np.int8), _c(w2, np.int8)
+    s13, s2 = _c(s13, np.float32), _c(s2, np.float32)
+    M, H = x.shape
+    I2, H2 = w13.shape
+    assert H2 == H and I2 % 2 == 0 and w2.shape == (H, I2 // 2)
+    I = I2 // 2
+    out = dict(y=np.empty((M, H), np.uint16), y32=np.empty((M, H), np.float32),
+               qx=np.empty((M, H), np.int8), sx=np.empty(M, np.float32),
+               qa=np.empty((M, I), np.int8), sa=np.empty(M, np.float32))
+    lib().oracle_mlp_forward(_p(x), _p(w13), _p(s13), _p(w2), _p(s2), M, H, I, _p(out["y"]), _p(out["y32"]),
+                             _p(out["qx"]), _p(out["sx"]), _p(out["qa"]), _p(out["sa"]))
     return out
 
 

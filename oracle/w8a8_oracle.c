@@ -411,6 +411,57 @@ void oracle_moe_forward(const bf16_t* x, const bf16_t* logits,
 }
 
 /* ------------------------------------------------------------------ */
+/* Dense gated MLP block (the dense analogue of a8-a10: [ATOM] "Changes": */
+/* gemm1 with fused gated-SiLU via interleaved w13 -> per-token int8     */
+/* quant -> gemm2).  For each token m:                                   */
+/*   (qx, sx) = quant_row(x[m])                                          */
+/*   v_r  = (float(sum_h qx[h] w13[r,h]) * sx) * s13[r],  r < 2I         */
+/*   a_i  = SiLU(v_2i) * v_2i+1;  (qa, sa) = quant_row(a)                */
+/*   y_n  = bf16( (float(sum_i qa[i] w2[n,i]) * sa) * s2[n] )            */
+/* w13 int8 [2I, H] (row 2i gate_i, 2i+1 up_i), s13 [2I]; w2 [H, I], s2 [H]. */
+void oracle_mlp_forward(const bf16_t* x, const int8_t* w13, const float* s13,
+                        const int8_t* w2, const float* s2, int64_t M, int H, int I,
+                        bf16_t* y, float* y32, int8_t* qx_out, float* sx_out,
+                        int8_t* qa_out, float* sa_out)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        float* xr = (float*)malloc(sizeof(float) * (size_t)H);
+        int8_t* qx = (int8_t*)malloc((size_t)H);
+        float* v = (float*)malloc(sizeof(float) * (size_t)(2 * I));
+        float* a = (float*)malloc(sizeof(float) * (size_t)I);
+        int8_t* qa = (int8_t*)malloc((size_t)I);
+        float sx, sa;
+        for (int h = 0; h < H; ++h) xr[h] = oracle_bf16_to_f32(x[m * H + h]);
+        oracle_quant_row_f32(xr, H, qx, &sx);
+        for (int r = 0; r < 2 * I; ++r) {
+            int64_t sum = 0;
+            for (int h = 0; h < H; ++h) sum += (int64_t)qx[h] * (int64_t)w13[(int64_t)r * H + h];
+            float vr = (float)(int32_t)sum;
+            vr = vr * sx;
+            vr = vr * s13[r];
+            v[r] = vr;
+        }
+        for (int i = 0; i < I; ++i) a[i] = oracle_silu(v[2 * i]) * v[2 * i + 1];
+        oracle_quant_row_f32(a, I, qa, &sa);
+        for (int n = 0; n < H; ++n) {
+            int64_t sum = 0;
+            for (int i = 0; i < I; ++i) sum += (int64_t)qa[i] * (int64_t)w2[(int64_t)n * I + i];
+            float y2 = (float)(int32_t)sum;
+            y2 = y2 * sa;
+            y2 = y2 * s2[n];
+            if (y) y[m * H + n] = oracle_f32_to_bf16(y2);
+            if (y32) y32[m * H + n] = y2;
+        }
+        if (qx_out) memcpy(qx_out + m * H, qx, (size_t)H);
+        if (sx_out) sx_out[m] = sx;
+        if (qa_out) memcpy(qa_out + m * I, qa, (size_t)I);
+        if (sa_out) sa_out[m] = sa;
+        free(xr); free(qx); free(v); free(a); free(qa);
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* a12: FWHT128 group quantization ([IQ8R] file table: "each 128 of K   */
 /* rotated by the unnormalised Hadamard", codes -127..127, a bf16 scale */
 /* per row and 128 of K; recipe: transform=fwht128 group=128 scale=bf16 */
