@@ -437,6 +437,31 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
                              "unit": "TOPS", "frac": ops / (t_gemm * 1e-3) / 1e12 / int8_peak,
                              "peak_source": "2 x measured bf16 burst (dense int8 : bf16 = 2 : 1)"}}
             del x, y, ws, qx, sx
+    # ---- dense gated MLP block: the same two matrices as gate_up (w13) and down (w2)
+    q13, s13 = W["gate_up"]
+    q2, s2 = W["down"]
+    I = q13.shape[0] // 2
+    H = q2.shape[0]
+    for M in (8, 4096):
+        x = bf16_dev(torch, inputs.dense_linear(9, M, H, 16, with_weights=False)[0], dev)
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.mlp_workspace_size(M, H, I), dtype=torch.uint8, device=dev)
+        fn = lambda: w8a8.mlp_forward(x, q13, s13, q2, s2, y=y, ws=ws)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        wbytes = q13.numel() + q2.numel() + 4 * (q13.shape[0] + H)
+        ops = 2.0 * M * (2 * I) * H + 2.0 * M * H * I
+        rec = {"ms": t, "weight_gbs": wbytes / (t * 1e-3) / 1e9, "tops": ops / (t * 1e-3) / 1e12}
+        if M == 8:
+            tg = graph_events(torch, fn, 10, flush=flush)
+            rec["graph_replay_ms"] = tg
+            rec["roofline"] = {"bound": "hbm", "frac": rec["weight_gbs"] / hbm, "peak": hbm, "unit": "GB/s",
+                               "bytes": wbytes}
+        else:
+            rec["roofline"] = {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"}
+        out[f"mlp_M{M}"] = rec
+        del x, y, ws
     # ---- per-token activation quant alone (a1) at the prefill shape
     for K in (5120, 17408):
         xq_in = bf16_dev(torch, inputs.dense_linear(5, 4096, K, 16, with_weights=False)[0], dev)

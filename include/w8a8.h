@@ -160,6 +160,31 @@ W8A8_API int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const i
                      void* ws, size_t ws_bytes, const w8a8_moe_debug* dbg, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Dense gated MLP block -- the dense analogue of a8 .. a10 ([ATOM] "Changes":
+ * gemm1 with fused gated SiLU over interleaved w13, per-token int8 quant,
+ * gemm2), one expert without routing:
+ *   x    bf16 [M, H];  w13 int8 [2I, H] (row 2i = gate_i, 2i+1 = up_i), s13 fp32 [2I]
+ *   w2   int8 [H, I];  s2 fp32 [H];   y bf16 [M, H]
+ * Steps: (qx, sx) = per-token quant of x; v = (float(qx . w13[r]) * sx) *
+ * s13[r]; a_i = SiLU(v_2i) * v_2i+1 (fp32, the project exponential);
+ * (qa, sa) = per-row quant of a; y = bf16( (float(qa . w2[n]) * sa) * s2[n] ).
+ * M <= 8 runs the weight-streaming GEMV path, larger M the tcgen05 GEMMs.
+ * Requires H % 16 == 0 and I % 16 == 0; 16-byte aligned pointers.
+ * ws_bytes >= w8a8_mlp_workspace_size(M, H, I).  `dbg` may be NULL;
+ * otherwise its non-NULL members receive intermediate values. */
+typedef struct w8a8_mlp_debug {
+    int8_t* qx;          /* [M, H] codes of x */
+    float* sx;           /* [M] */
+    int8_t* qa;          /* [M, I] codes of the gated intermediate */
+    float* sa;           /* [M] */
+} w8a8_mlp_debug;
+
+W8A8_API size_t w8a8_mlp_workspace_size(int64_t M, int64_t H, int64_t I);
+W8A8_API int w8a8_mlp_forward(const uint16_t* x, const int8_t* w13, const float* s13, const int8_t* w2,
+                              const float* s2, uint16_t* y, int64_t M, int64_t H, int64_t I, void* ws,
+                              size_t ws_bytes, const w8a8_mlp_debug* dbg, void* stream);
+
+/* ---------------------------------------------------------------------------
  * FWHT128-domain group quantization (a12) -- [IQ8R] file table ("each 128 of
  * K rotated by the unnormalised Hadamard"; codes -127..127; a bf16 scale per
  * row and 128 of K) and recipe (transform=fwht128 group=128 scale=bf16

@@ -96,7 +96,7 @@ __device__ __forceinline__ void tc2_commit_pair(uint64_t* bar) {
 template <int EPI>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
-    static_assert(EPI == kEpiBf16 || EPI == kEpiS32, "dense epilogues");
+    static_assert(EPI == kEpiBf16 || EPI == kEpiS32 || EPI == kEpiMoeGated, "dense epilogues");
     constexpr int kCols = 2 * kTc2BN;   // two accumulators of 256 columns
     using SM = Tc2Smem;
     extern __shared__ uint8_t smem_raw[];
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
             const int row = mt * kTc2BM + (int)rank * 128 + quarter * 32 + lane;
             const bool row_ok = row < p.M;
             float sxr = 0.0f;
-            if (EPI == kEpiBf16 && row_ok) sxr = __ldg(p.sx + row);
+            if ((EPI == kEpiBf16 || EPI == kEpiMoeGated) && row_ok) sxr = __ldg(p.sx + row);
             const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kTc2BN);
 #pragma unroll 1
             for (int c = 0; c < kTc2BN; c += 32) {
@@ -266,6 +266,23 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                             }
                             *reinterpret_cast<uint4*>(yrow + n0 + v * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
+                    }
+                } else if (EPI == kEpiMoeGated) {
+                    // columns n0 .. n0+31: 16 (gate, up) pairs -> a[row, n0/2 .. n0/2+15] (N % 32 == 0)
+                    const float* swc = p.sw + n0;
+                    float* arow = p.a_out + (int64_t)row * (p.N / 2) + n0 / 2;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float av[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int j = 8 * q + 2 * i;
+                            const float vg = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), __ldg(swc + j));
+                            const float vu =
+                                __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sxr), __ldg(swc + j + 1));
+                            av[i] = __fmul_rn(silu_proj(vg), vu);
+                        }
+                        *reinterpret_cast<float4*>(arow + 4 * q) = make_float4(av[0], av[1], av[2], av[3]);
                     }
                 } else {
                     int32_t* orow = reinterpret_cast<int32_t*>(p.out) + (int64_t)row * p.N;

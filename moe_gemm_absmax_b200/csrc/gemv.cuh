@@ -246,6 +246,43 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_dense_kernel(GemvShap
 }
 
 
+// ---------------------------------------------------------------- gated
+// The gate_up projection of a dense gated MLP: weight rows 2i (gate) and
+// 2i + 1 (up) interleaved; RowMapPairs puts gate row 2(8b + g) in MMA row g
+// and its up row in MMA row g + 8 of the same lane, so each thread holds
+// (gate, up) of one pair for tokens 2t and 2t + 1:
+//   v = (float(acc) * sx[m]) * sw[row];  a[m, i] = SiLU(v_gate) * v_up  (fp32)
+struct GemvEpiGated {
+    const float* sx;   // [M]
+    const float* sw;   // [2I]
+    float* a;          // [M, I]
+    int M, I;
+};
+
+template <int WN, int WK, int TG, int U, int MINB = 1>
+__global__ void __launch_bounds__(kGemvThreads, MINB) gemv_gated_kernel(GemvShape a, GemvEpiGated e) {
+    int acc[TG][4];
+    int block;
+    if (!gemv_core<WN, WK, TG, RowMapPairs, U>(a, acc, block, blockIdx.y, gridDim.y, blockIdx.x)) return;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int pair = block * 8 + g;
+    if (pair >= e.I) return;
+    const float swg = __ldg(e.sw + 2 * pair), swu = __ldg(e.sw + 2 * pair + 1);
+#pragma unroll
+    for (int tg = 0; tg < TG; ++tg) {
+#pragma unroll
+        for (int jt = 0; jt < 2; ++jt) {
+            const int m = tg * 8 + 2 * t + jt;
+            if (m < e.M) {
+                const float sxm = __ldcg(e.sx + m);
+                const float vg = __fmul_rn(__fmul_rn(__int2float_rn(acc[tg][jt]), sxm), swg);
+                const float vu = __fmul_rn(__fmul_rn(__int2float_rn(acc[tg][2 + jt]), sxm), swu);
+                e.a[(int64_t)m * e.I + pair] = __fmul_rn(silu_proj(vg), vu);
+            }
+        }
+    }
+}
+
 }  // namespace w8a8
 
 

@@ -285,6 +285,34 @@ int launch_gemv_reg(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g
     return cuda_status(cudaLaunchKernelEx(&cfg, gemv_dense_kernel<kGemvWN, kGemvWK, TG, U, kGemvMinBlocks>, a, e));
 }
 
+// gate_up GEMV of the dense MLP block, gated epilogue (same plan as the dense GEMV).
+int launch_gemv_gated(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, float* a_out, int64_t M,
+                      int64_t I, int64_t K, const GemvPlan& g, void* scratch, bool after_quant, cudaStream_t st) {
+    GemvShape a;
+    a.w = qw;
+    a.x = qx;
+    a.tokens = (int)M;
+    a.rows = (int)(2 * I);
+    a.K = (int)K;
+    a.nchunks = (int)((K + 63) / 64);
+    a.part = reinterpret_cast<int32_t*>(scratch);
+    a.counters = gemv_counters(g, scratch);
+    GemvEpiGated e;
+    e.sx = sx;
+    e.sw = sw;
+    e.a = a_out;
+    e.M = (int)M;
+    e.I = (int)I;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.ctas_x, (unsigned)g.nkseg, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    pdl_config(cfg, at, after_quant);
+    return cuda_status(
+        cudaLaunchKernelEx(&cfg, gemv_gated_kernel<kGemvWN, kGemvWK, 1, kGemvUnrollDecode, kGemvMinBlocks>, a, e));
+}
+
 // Runs the GEMV; `scratch` holds the partials and the counters (zero on entry).
 int run_gemv(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, void* out, int64_t M, int64_t N,
              int64_t K, bool s32, const GemvPlan& g, void* scratch, bool after_quant, cudaStream_t st) {
@@ -417,6 +445,43 @@ MoeWs moe_carve(void* base, int64_t T, int E, int H, int I, int topk) {
     w.sa = reinterpret_cast<float*>(take((size_t)R * 4));
     // w * y2 at (token, slot), or the atomically combined [T, H] for large T
     w.out = reinterpret_cast<float*>(take(moe_exact_combine(R, H) ? (size_t)R * H * 4 : (size_t)T * H * 4));
+    w.bytes = o;
+    return w;
+}
+
+// Dense gated MLP block workspace: x codes and scales, the fp32 gated
+// intermediate, its codes and scales, and (decode) the two GEMVs' split-K
+// partials and counters.
+struct MlpWs {
+    int8_t* qx;
+    float* sx;
+    float* a;
+    int8_t* qa;
+    float* sa;
+    void* scratch1;
+    void* scratch2;
+    size_t bytes;
+};
+
+MlpWs mlp_carve(void* base, int64_t M, int64_t H, int64_t I) {
+    MlpWs w;
+    uint8_t* p = reinterpret_cast<uint8_t*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* r = p ? p + o : nullptr;
+        o += align_up(bytes, 256);
+        return r;
+    };
+    w.qx = reinterpret_cast<int8_t*>(take((size_t)(M * H)));
+    w.sx = reinterpret_cast<float*>(take((size_t)M * 4));
+    w.a = reinterpret_cast<float*>(take((size_t)(M * I) * 4));
+    w.qa = reinterpret_cast<int8_t*>(take((size_t)(M * I)));
+    w.sa = reinterpret_cast<float*>(take((size_t)M * 4));
+    w.scratch1 = w.scratch2 = nullptr;
+    if (M <= 8) {
+        w.scratch1 = take(gemv_ws_bytes(gemv_plan(M, 2 * I, H)));
+        w.scratch2 = take(gemv_ws_bytes(gemv_plan(M, H, I)));
+    }
     w.bytes = o;
     return w;
 }
@@ -853,6 +918,70 @@ int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w1
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
 
     return moe_debug_copies(w, dbg, R, E, I, st);
+}
+
+// ----------------------------------------------------------------- dense gated MLP block
+size_t w8a8_mlp_workspace_size(int64_t M, int64_t H, int64_t I) {
+    if (M <= 0 || H <= 0 || I <= 0) return 0;
+    return mlp_carve(nullptr, M, H, I).bytes;
+}
+
+int w8a8_mlp_forward(const uint16_t* x, const int8_t* w13, const float* s13, const int8_t* w2, const float* s2,
+                     uint16_t* y, int64_t M, int64_t H, int64_t I, void* ws, size_t ws_bytes,
+                     const w8a8_mlp_debug* dbg, void* stream) {
+    if (!x || !w13 || !s13 || !w2 || !s2 || !y || !ws) return W8A8_ERR_INVALID_ARG;
+    if (M <= 0 || H <= 0 || I <= 0 || H % 16 != 0 || I % 16 != 0) return W8A8_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(M, 2 * I, H) || !gemm_shape_ok(M, H, I)) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w13, 16) || !aligned(s13, 16) || !aligned(w2, 16) || !aligned(s2, 16) ||
+        !aligned(y, 16) || !aligned(ws, 256))
+        return W8A8_ERR_INVALID_ARG;
+    if (H / 8 > (int64_t)8 * 256 * kQuantMaxVec || I / 4 > (int64_t)8 * 256 * kQuantMaxVec) return W8A8_ERR_UNSUPPORTED;
+    if (ws_bytes < w8a8_mlp_workspace_size(M, H, I)) return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const MlpWs w = mlp_carve(ws, M, H, I);
+    const bool gemv = M <= 8;
+    const GemvPlan g1 = gemv_plan(M, 2 * I, H), g2 = gemv_plan(M, H, I);
+    int* ctr1 = gemv ? gemv_counters(g1, w.scratch1) : nullptr;
+    int* ctr2 = gemv ? gemv_counters(g2, w.scratch2) : nullptr;
+    int rc;
+    // a1 (it also clears the gate_up GEMV's counters)
+    if (launch_quant_rows<uint16_t>(x, M, H, H, w.qx, H, w.sx, st, current_sms(), ctr1, ctr1 ? g1.counters : 0) !=
+        cudaSuccess)
+        return W8A8_ERR_CUDA;
+    // gate_up GEMM with SiLU(gate) * up -> fp32 a [M, I]
+    if (gemv) {
+        rc = launch_gemv_gated(w.qx, w.sx, w13, s13, w.a, M, I, H, g1, w.scratch1, true, st);
+    } else {
+        TcParams p = {};
+        p.M = (int)M;
+        p.N = (int)(2 * I);
+        p.K = (int)H;
+        p.sx = w.sx;
+        p.sw = s13;
+        p.a_out = w.a;
+        rc = M >= kTc2MinM ? launch_tc2<kEpiMoeGated>(w.qx, w13, p, st)
+                           : launch_tc<256, 4, kEpiMoeGated, 2, 8>(w.qx, w13, p, st);
+    }
+    if (rc != W8A8_OK) return rc;
+    // a9 (it also clears the down GEMV's counters)
+    if (launch_quant_rows<float>(w.a, M, I, I, w.qa, I, w.sa, st, current_sms(), ctr2, ctr2 ? g2.counters : 0) !=
+        cudaSuccess)
+        return W8A8_ERR_CUDA;
+    // down GEMM with the dense dequant
+    rc = gemv ? run_gemv(w.qa, w.sa, w2, s2, y, M, H, I, false, g2, w.scratch2, true, st)
+              : run_tc(w.qa, w.sa, w2, s2, y, M, H, I, kEpiBf16, st);
+    if (rc != W8A8_OK) return rc;
+    if (dbg) {
+        if (dbg->qx && cudaMemcpyAsync(dbg->qx, w.qx, (size_t)(M * H), cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->sx && cudaMemcpyAsync(dbg->sx, w.sx, (size_t)M * 4, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->qa && cudaMemcpyAsync(dbg->qa, w.qa, (size_t)(M * I), cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->sa && cudaMemcpyAsync(dbg->sa, w.sa, (size_t)M * 4, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+    }
+    return W8A8_OK;
 }
 
 // ----------------------------------------------------------------- FWHT128

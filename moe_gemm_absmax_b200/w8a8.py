@@ -24,7 +24,8 @@ EXPORTS = (
     "w8a8_quant_act", "w8a8_quant_rows_f32", "w8a8_linear_workspace_size", "w8a8_linear",
     "w8a8_linear_noalloc_scratch_size", "w8a8_linear_noalloc",
     "w8a8_gemm_workspace_size", "w8a8_gemm_q", "w8a8_gemm_s32", "w8a8_moe_workspace_size",
-    "w8a8_moe_forward", "fwht128_quant", "w8a8_linear_g128", "w8a8_exp_proj",
+    "w8a8_moe_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
+    "w8a8_exp_proj",
     "w8a8_get_device_error", "w8a8_debug_wait_timeout", "w8a8_status_str", "w8a8_version",
 )
 
@@ -35,6 +36,10 @@ class W8A8Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+class MlpDebug(ctypes.Structure):
+    _fields_ = [("qx", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("qa", ctypes.c_void_p), ("sa", ctypes.c_void_p)]
 
 
 class MoeDebug(ctypes.Structure):
@@ -65,6 +70,8 @@ def lib() -> ctypes.CDLL:
         "w8a8_moe_workspace_size": ([i64, i32, i32, i32, i32], sz),
         "w8a8_moe_forward": ([vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, sz,
                               ctypes.POINTER(MoeDebug), vp], i32),
+        "w8a8_mlp_workspace_size": ([i64, i64, i64], sz),
+        "w8a8_mlp_forward": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, ctypes.POINTER(MlpDebug), vp], i32),
         "fwht128_quant": ([vp, i64, i64, vp, vp, vp], i32),
         "w8a8_linear_g128": ([vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "w8a8_exp_proj": ([vp, vp, i64, vp], i32),
@@ -266,6 +273,40 @@ def moe_forward(x, logits, w13, s13, w2, s2, topk: int = 8, y=None, ws=None, deb
     _check(lib().w8a8_moe_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13), _ptr(w2), _ptr(s2), _ptr(y),
                                   T, E, H, I, topk, _ptr(ws), ws.numel(), dbg_p, _stream(stream)),
            "w8a8_moe_forward")
+    return (y, dbg_t) if debug else y
+
+
+# ------------------------------------------------------------------ dense gated MLP block
+
+def mlp_workspace_size(M: int, H: int, I: int) -> int:
+    return int(lib().w8a8_mlp_workspace_size(M, H, I))
+
+
+def mlp_forward(x, w13, s13, w2, s2, y=None, ws=None, debug: bool = False, stream=None):
+    """Dense gated MLP block: bf16 x [M,H] -> gate_up (w13 int8 [2I,H], rows 2i gate /
+    2i+1 up, s13 [2I]) with SiLU(gate)*up -> requant -> down (w2 int8 [H,I], s2 [H])
+    -> bf16 y [M,H].  Returns y, or (y, debug dict) when debug."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w13, torch.int8, "w13", 2)
+    _need(w2, torch.int8, "w2", 2)
+    _need(s13, torch.float32, "s13", 1)
+    _need(s2, torch.float32, "s2", 1)
+    M, H = x.shape
+    I = w13.shape[0] // 2
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = _workspace(mlp_workspace_size(M, H, I), dev)
+    dbg_t = dbg_p = None
+    if debug:
+        dbg_t = dict(qx=torch.empty((M, H), dtype=torch.int8, device=dev),
+                     sx=torch.empty(M, dtype=torch.float32, device=dev),
+                     qa=torch.empty((M, I), dtype=torch.int8, device=dev),
+                     sa=torch.empty(M, dtype=torch.float32, device=dev))
+        dbg_p = ctypes.pointer(MlpDebug(*[v.data_ptr() for v in dbg_t.values()]))
+    _check(lib().w8a8_mlp_forward(_ptr(x), _ptr(w13), _ptr(s13), _ptr(w2), _ptr(s2), _ptr(y), M, H, I, _ptr(ws),
+                                  ws.numel(), dbg_p, _stream(stream)), "w8a8_mlp_forward")
     return (y, dbg_t) if debug else y
 
 
