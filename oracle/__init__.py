@@ -80,6 +80,9 @@ def lib():
             L.oracle_fwht128.argtypes = [vp]
             L.oracle_fwht128_quant.argtypes = [vp, i64, i64, vp, vp, vp]
             L.oracle_gemm_g128.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
+            L.oracle_fwht128_quant_f32.argtypes = [vp, i64, i64, vp, vp]
+            L.oracle_moe_g128_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32,
+                                                  vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.oracle_set_threads.argtypes = [i32]
             L.oracle_get_threads.restype = i32
         return _lib
@@ -282,6 +285,48 @@ def fwht128_quant(x_bits):
     xr = np.empty((M, K), np.float32)
     lib().oracle_fwht128_quant(_p(x), M, K, _p(q), _p(s), _p(xr))
     return q, s, xr
+
+
+def fwht128_quant_f32(x):
+    """a12 on fp32 rows: returns (codes int8 [M,K], scales bf16 bits [M,K/128])."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    assert K % 128 == 0
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M, K // 128), np.uint16)
+    lib().oracle_fwht128_quant_f32(_p(x), M, K, _p(q), _p(s))
+    return q, s
+
+
+def moe_g128_forward(x_bits, logits_bits, w13, s13_bits, w2, s2_bits, topk: int, tokens=None):
+    """Routed experts on the FWHT128 grid for the listed tokens (all when
+    None).  w13 int8 [E,2I,H] + bf16 bits [E,2I,H/128]; w2 int8 [E,H,I] +
+    bf16 bits [E,H,I/128].  Returns a dict like moe_forward, with the scales
+    sx [n,H/128] and sa [n,k,I/128] as bf16 bits."""
+    x = _c(x_bits, np.uint16)
+    lg = _c(logits_bits, np.uint16)
+    w13, w2 = _c(w13, np.int8), _c(w2, np.int8)
+    s13, s2 = _c(s13_bits, np.uint16), _c(s2_bits, np.uint16)
+    T, H = x.shape
+    E, I2, H2 = w13.shape
+    assert H2 == H and I2 % 2 == 0 and H % 128 == 0
+    I = I2 // 2
+    assert I % 128 == 0 and w2.shape == (E, H, I)
+    assert s13.shape == (E, I2, H // 128) and s2.shape == (E, H, I // 128)
+    toks = np.arange(T, dtype=np.int64) if tokens is None else _c(tokens, np.int64)
+    n = toks.size
+    out = dict(
+        y=np.empty((n, H), np.uint16), y32=np.empty((n, H), np.float32),
+        yabs=np.empty((n, H), np.float32), ids=np.empty((n, topk), np.int32),
+        wts=np.empty((n, topk), np.float32), qx=np.empty((n, H), np.int8),
+        sx=np.empty((n, H // 128), np.uint16), qa=np.empty((n, topk, I), np.int8),
+        sa=np.empty((n, topk, I // 128), np.uint16))
+    lib().oracle_moe_g128_forward(_p(x), _p(lg), _p(w13), _p(s13), _p(w2), _p(s2), T, E, H, I, topk,
+                                  _p(toks), n, _p(out["y"]), _p(out["y32"]), _p(out["yabs"]),
+                                  _p(out["ids"]), _p(out["wts"]), _p(out["qx"]), _p(out["sx"]),
+                                  _p(out["qa"]), _p(out["sa"]))
+    out["tokens"] = toks
+    return out
 
 
 def gemm_g128(qx, sx_bits, qw, sw_bits):

@@ -485,6 +485,23 @@ void oracle_fwht128(float* v)
     }
 }
 
+/* One 128-wide block already in fp32: rotate it in place, then the bf16  */
+/* scale and the codes from that stored scale.                           */
+static bf16_t fwht128_quant_block(float* v, int8_t* q)
+{
+    oracle_fwht128(v);
+    float amax = 0.0f;
+    for (int k = 0; k < 128; ++k) { float a = fabsf(v[k]); if (a > amax) amax = a; }
+    bf16_t sb = oracle_f32_to_bf16(amax / 127.0f);
+    float sf = oracle_bf16_to_f32(sb);
+    for (int k = 0; k < 128; ++k) {
+        int8_t code = 0;
+        if (sf != 0.0f) code = clamp_sym127(rne_to_int(v[k] / sf));
+        q[k] = code;
+    }
+    return sb;
+}
+
 void oracle_fwht128_quant(const bf16_t* x, int64_t M, int64_t K, int8_t* q, bf16_t* s,
                           float* xr_out)
 {
@@ -494,18 +511,22 @@ void oracle_fwht128_quant(const bf16_t* x, int64_t M, int64_t K, int8_t* q, bf16
         float v[128];
         for (int64_t g = 0; g < G; ++g) {
             for (int k = 0; k < 128; ++k) v[k] = oracle_bf16_to_f32(x[m * K + g * 128 + k]);
-            oracle_fwht128(v);
+            s[m * G + g] = fwht128_quant_block(v, q + m * K + g * 128);
             if (xr_out) for (int k = 0; k < 128; ++k) xr_out[m * K + g * 128 + k] = v[k];
-            float amax = 0.0f;
-            for (int k = 0; k < 128; ++k) { float a = fabsf(v[k]); if (a > amax) amax = a; }
-            bf16_t sb = oracle_f32_to_bf16(amax / 127.0f);
-            float sf = oracle_bf16_to_f32(sb);
-            s[m * G + g] = sb;
-            for (int k = 0; k < 128; ++k) {
-                int8_t code = 0;
-                if (sf != 0.0f) code = clamp_sym127(rne_to_int(v[k] / sf));
-                q[m * K + g * 128 + k] = code;
-            }
+        }
+    }
+}
+
+/* The same for fp32 rows (the routed experts' gated intermediate). */
+void oracle_fwht128_quant_f32(const float* x, int64_t M, int64_t K, int8_t* q, bf16_t* s)
+{
+    int64_t G = K / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        float v[128];
+        for (int64_t g = 0; g < G; ++g) {
+            for (int k = 0; k < 128; ++k) v[k] = x[m * K + g * 128 + k];
+            s[m * G + g] = fwht128_quant_block(v, q + m * K + g * 128);
         }
     }
 }
@@ -536,6 +557,101 @@ void oracle_gemm_g128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, cons
             if (y) y[m * N + n] = oracle_f32_to_bf16(r);
             if (y32) y32[m * N + n] = r;
         }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* f1: routed experts on the rotated grid ([IQ8R] file table: "Experts   */
+/* ... int8 on the same rotated grid with a bf16 scale per row and 128  */
+/* of K"; "Activations int8 under the same rotation, the routed experts  */
+/* reading the codes the trunk's quantisers write"; recipe rows          */
+/* ffn_gate_up_exps / ffn_down_exps: group=128 scale=bf16                 */
+/* transform=fwht128).  The pipeline is that of oracle_moe_forward with  */
+/* each quantizer replaced by the FWHT128 group quantizer and each GEMM  */
+/* by the group-128 GEMM of oracle_gemm_g128.  Per token t and slot j    */
+/* (expert e = ids[t,j]):                                                 */
+/*   (qx, sx[g]) = fwht128_quant(x[t])           (rotation along H)       */
+/*   v_r  = g128(qx, sx; w13[e,r], s13[e,r])     (fp32, not rounded)      */
+/*   a_i  = SiLU(v_2i) * v_2i+1                                           */
+/*   (qa, sa[g]) = fwht128_quant(a)              (rotation along I, fp32) */
+/*   y2_n = g128(qa, sa; w2[e,n], s2[e,n])                                */
+/*   out_n = sum over j = 0..k-1 of wts[t,j] * y2_n   (fp32, slot order)  */
+/* with g128(qa, sa; qw, sw) = (sum over g ascending of                   */
+/*   fma(float(p_g), float(sa[g]) * float(sw[g]), acc)) * (1/128).        */
+/* w13 int8 [E, 2I, H] + bf16 [E, 2I, H/128]; w2 int8 [E, H, I] + bf16    */
+/* [E, H, I/128] (rows rotated along K and group-quantized).              */
+/* Outputs per listed token as in oracle_moe_forward, with the scales    */
+/* bf16: sx [ntok, H/128], sa [ntok, k, I/128].                           */
+/* ------------------------------------------------------------------ */
+static float g128_dot(const int8_t* qa, const bf16_t* sa, const int8_t* qw, const bf16_t* sw, int64_t K)
+{
+    float acc = 0.0f;
+    for (int64_t g = 0; g < K / 128; ++g) {
+        int32_t p = 0;
+        for (int k = 0; k < 128; ++k) p += (int32_t)qa[g * 128 + k] * (int32_t)qw[g * 128 + k];
+        float sc = oracle_bf16_to_f32(sa[g]) * oracle_bf16_to_f32(sw[g]);
+        acc = fmaf((float)p, sc, acc);
+    }
+    return acc * 0.0078125f;
+}
+
+void oracle_moe_g128_forward(const bf16_t* x, const bf16_t* logits,
+                             const int8_t* w13, const bf16_t* s13,
+                             const int8_t* w2, const bf16_t* s2,
+                             int64_t T, int E, int H, int I, int topk,
+                             const int64_t* toks, int64_t ntok,
+                             bf16_t* y, float* y32, float* yabs,
+                             int32_t* ids_out, float* wts_out,
+                             int8_t* qx_out, bf16_t* sx_out,
+                             int8_t* qa_out, bf16_t* sa_out)
+{
+    (void)T;
+    const int GH = H / 128, GI = I / 128;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < ntok; ++i) {
+        int64_t t = toks[i];
+        int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)topk);
+        float* wts = (float*)malloc(sizeof(float) * (size_t)topk);
+        int8_t* qx = (int8_t*)malloc((size_t)H);
+        bf16_t* sx = (bf16_t*)malloc(sizeof(bf16_t) * (size_t)GH);
+        float* v = (float*)malloc(sizeof(float) * (size_t)(2 * I));
+        float* a = (float*)malloc(sizeof(float) * (size_t)I);
+        int8_t* qa = (int8_t*)malloc((size_t)I);
+        bf16_t* sa = (bf16_t*)malloc(sizeof(bf16_t) * (size_t)GI);
+        float* out = (float*)calloc((size_t)H, sizeof(float));
+        float* oabs = (float*)calloc((size_t)H, sizeof(float));
+
+        oracle_route(logits + t * E, 1, E, topk, ids, wts);
+        oracle_fwht128_quant(x + t * H, 1, H, qx, sx, NULL);
+
+        for (int j = 0; j < topk; ++j) {
+            int e = ids[j];
+            for (int r = 0; r < 2 * I; ++r) {
+                int64_t wr = (int64_t)e * 2 * I + r;
+                v[r] = g128_dot(qx, sx, w13 + wr * H, s13 + wr * GH, H);
+            }
+            for (int ii = 0; ii < I; ++ii) a[ii] = oracle_silu(v[2 * ii]) * v[2 * ii + 1];
+            oracle_fwht128_quant_f32(a, 1, I, qa, sa);
+            if (qa_out) memcpy(qa_out + (i * topk + j) * I, qa, (size_t)I);
+            if (sa_out) memcpy(sa_out + (i * topk + j) * GI, sa, sizeof(bf16_t) * (size_t)GI);
+            for (int n = 0; n < H; ++n) {
+                int64_t wr = (int64_t)e * H + n;
+                float y2 = g128_dot(qa, sa, w2 + wr * I, s2 + wr * GI, I);
+                float c = wts[j] * y2;
+                out[n] = out[n] + c;
+                oabs[n] = oabs[n] + fabsf(c);
+            }
+        }
+        for (int n = 0; n < H; ++n) {
+            if (y) y[i * H + n] = oracle_f32_to_bf16(out[n]);
+            if (y32) y32[i * H + n] = out[n];
+            if (yabs) yabs[i * H + n] = oabs[n];
+        }
+        if (ids_out) memcpy(ids_out + i * topk, ids, sizeof(int32_t) * (size_t)topk);
+        if (wts_out) memcpy(wts_out + i * topk, wts, sizeof(float) * (size_t)topk);
+        if (qx_out) memcpy(qx_out + i * H, qx, (size_t)H);
+        if (sx_out) memcpy(sx_out + i * GH, sx, sizeof(bf16_t) * (size_t)GH);
+        free(ids); free(wts); free(qx); free(sx); free(v); free(a); free(qa); free(sa); free(out); free(oabs);
     }
 }
 
