@@ -478,6 +478,9 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
     w13, w2 = inputs.moe_weights(0)
     q13, s13 = quantize_on_gpu(torch, w8a8, w13, dev)
     q2, s2 = quantize_on_gpu(torch, w8a8, w2, dev)
+    # the same experts on the FWHT128 grid (bf16 rows rotated along K, group codes)
+    g13 = w8a8.fwht128_quant(bf16_dev(torch, inputs.to_bf16_bits(w13).reshape(-1, w13.shape[2]), dev))
+    g2 = w8a8.fwht128_quant(bf16_dev(torch, inputs.to_bf16_bits(w2).reshape(-1, w2.shape[2]), dev))
     del w13, w2
     E, I2, H = q13.shape
     per_expert = q13[0].numel() + q2[0].numel() + 4 * (I2 + H)
@@ -501,6 +504,30 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
                                          "bytes": byts}}
         del x, lg, y, ws
     del q13, q2
+    # ---- routed MoE layer on the FWHT128 grid
+    gq13, gs13 = g13[0].view(E, I2, H), g13[1].view(E, I2, H // 128)
+    gq2, gs2 = g2[0].view(E, H, I2 // 2), g2[1].view(E, H, I2 // 256)
+    per_expert = gq13[0].numel() + gq2[0].numel() + 2 * (gs13[0].numel() + gs2[0].numel())
+    for T in (1, 8, 512, 4096):
+        xb, lb = inputs.moe_tokens(0, T)
+        x, lg = bf16_dev(torch, xb, dev), bf16_dev(torch, lb, dev)
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.moe_g128_workspace_size(T, E, H, I2 // 2, 8), dtype=torch.uint8, device=dev)
+        fn = lambda: w8a8.moe_g128_forward(x, lg, gq13, gs13, gq2, gs2, 8, y=y, ws=ws)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        tg = graph_events(torch, fn, 10, flush=flush)
+        _, dbg = w8a8.moe_g128_forward(x, lg, gq13, gs13, gq2, gs2, 8, debug=True)
+        touched = int((dbg["counts"] > 0).sum().item())
+        byts = touched * per_expert + 2 * T * H * 2 + 2 * T * E
+        out[f"moe_g128_T{T}"] = {"ms": t, "tokens_per_s": T / (t * 1e-3), "touched_experts": touched,
+                                 "graph_replay_ms": tg, "graph_replay_tokens_per_s": T / (tg * 1e-3),
+                                 "roofline": {"bound": "hbm", "achieved": byts / (t * 1e-3) / 1e9, "peak": hbm,
+                                              "unit": "GB/s", "frac": byts / (t * 1e-3) / 1e9 / hbm,
+                                              "bytes": byts}}
+        del x, lg, y, ws
+    del g13, g2, gq13, gs13, gq2, gs2
     # ---- FWHT128-domain linear
     _, wb = inputs.hadamard_linear(0, 1)
     qw, sw = w8a8.fwht128_quant(bf16_dev(torch, wb, dev))
@@ -531,7 +558,8 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
 # --------------------------------------------------------------------------- profiling cases
 CASES = ("gemv_gateup_m8", "gemv_down_m8", "prefill_gateup_m512", "prefill_down_m512", "prefill_gateup_m4096",
          "prefill_down_m4096", "quant_m4096_k17408", "quant_m4096_k5120", "moe_t1", "moe_t8", "moe_t512",
-         "moe_t4096", "hadamard_m1", "hadamard_m200", "hadamard_m2048")
+         "moe_t4096", "moe_g128_t1", "moe_g128_t8", "moe_g128_t512", "moe_g128_t4096", "hadamard_m1",
+         "hadamard_m200", "hadamard_m2048")
 
 
 def run_case(name, torch, dev, reps=4):
@@ -546,6 +574,8 @@ def run_case(name, torch, dev, reps=4):
         return torch.randn(*shape, generator=g, device=dev) * std
 
     kind, _, rest = name.partition("_")
+    if name.startswith("moe_g128_"):
+        kind, rest = "moe_g128", name[len("moe_g128_"):]
     if kind in ("gemv", "prefill"):
         which, m = rest.split("_")
         d = inputs.GATE_UP if which == "gateup" else inputs.DOWN
@@ -574,6 +604,20 @@ def run_case(name, torch, dev, reps=4):
         torch.cuda.empty_cache()
         for _ in range(reps):
             w8a8.moe_forward(x, lg, q13, s13, q2, s2, k, y=y, ws=ws)
+    elif kind == "moe_g128":
+        T = int(rest[1:])
+        E, H, I, k = inputs.MOE["E"], inputs.MOE["H"], inputs.MOE["I"], inputs.MOE["topk"]
+        q13, s13 = w8a8.fwht128_quant(randn(E * 2 * I, H, std=0.02).to(torch.bfloat16))
+        q2, s2 = w8a8.fwht128_quant(randn(E * H, I, std=0.02).to(torch.bfloat16))
+        q13, s13 = q13.view(E, 2 * I, H), s13.view(E, 2 * I, H // 128)
+        q2, s2 = q2.view(E, H, I), s2.view(E, H, I // 128)
+        x = randn(T, H).to(torch.bfloat16)
+        lg = randn(T, E).to(torch.bfloat16)
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.moe_g128_workspace_size(T, E, H, I, k), dtype=torch.uint8, device=dev)
+        torch.cuda.empty_cache()
+        for _ in range(reps):
+            w8a8.moe_g128_forward(x, lg, q13, s13, q2, s2, k, y=y, ws=ws)
     elif kind == "hadamard":
         M = int(rest[1:])
         d = inputs.HADAMARD

@@ -205,6 +205,47 @@ W8A8_API int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t
                      int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Routed experts on the FWHT128 grid -- [IQ8R] file table (Experts: int8 on
+ * the same rotated grid with a bf16 scale per row and 128 of K; Activations:
+ * int8 under the same rotation, the routed experts reading the codes the
+ * trunk's quantisers write) and recipe (ffn_gate_up_exps / ffn_down_exps:
+ * group=128 scale=bf16 transform=fwht128).  The layer of w8a8_moe_forward
+ * with each quantizer replaced by fwht128_quant and each expert GEMM by its
+ * group-128 form:
+ *   x       bf16 [T, H]             token activations (unrotated)
+ *   logits  bf16 [T, E]             router logits
+ *   w13     int8 [E, 2I, H]         rows rotated along H (fwht128_quant of the
+ *                                   bf16 rows), row 2i = gate_i, 2i+1 = up_i
+ *   s13     bf16 [E, 2I, H/128]
+ *   w2      int8 [E, H, I]          rows rotated along I; s2 bf16 [E, H, I/128]
+ *   y       bf16 [T, H]
+ * Steps: routing as w8a8_moe_forward; (qx, sx) = fwht128_quant(x[t]);
+ * v_r = (sum over g ascending of fma(float(p_g), sx[g] * s13[e,r,g], .)) / 128
+ * (fp32, p_g the int32 dot product of group g); a_i = SiLU(v_2i) * v_2i+1;
+ * (qa, sa) = FWHT128 group quant of the fp32 row a (rotated along I);
+ * y2_n = the same group-128 product of (qa, sa) with (w2[e,n], s2[e,n]);
+ * y = bf16( sum_j w_j * y2 ) with the k contributions added in fp32 in slot
+ * order.  Requires H % 128 == 0, H <= 4096, I % 128 == 0, I <= 2048,
+ * E <= 256, topk <= 32; 16-byte aligned x, w13, w2, y; 256-byte aligned ws.
+ * ws_bytes >= w8a8_moe_g128_workspace_size(T, E, H, I, topk).  `dbg` may be
+ * NULL; otherwise its non-NULL members receive intermediate values. */
+typedef struct w8a8_moe_g128_debug {
+    int32_t* topk_ids;   /* [T, topk], descending logits */
+    float* topk_w;       /* [T, topk] */
+    int32_t* counts;     /* [E] rows routed to each expert */
+    int8_t* qx;          /* [T, H] rotated codes of x */
+    uint16_t* sx;        /* [T, H/128] bf16 */
+    int8_t* qa;          /* [T, topk, I] rotated codes of the gated intermediate, by (token, slot) */
+    uint16_t* sa;        /* [T, topk, I/128] bf16 */
+} w8a8_moe_g128_debug;
+
+W8A8_API size_t w8a8_moe_g128_workspace_size(int64_t T, int E, int H, int I, int topk);
+W8A8_API int w8a8_moe_g128_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w13,
+                                   const uint16_t* s13, const int8_t* w2, const uint16_t* s2, uint16_t* y, int64_t T,
+                                   int E, int H, int I, int topk, void* ws, size_t ws_bytes,
+                                   const w8a8_moe_g128_debug* dbg, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics. */
 
 /* The library's fp32 exponential (Cody & Waite reduction, degree-7 Taylor),

@@ -169,6 +169,13 @@ __device__ __forceinline__ void tmem_st_32x32b_x32_fill(uint32_t taddr, uint32_t
                      "r"(v)
                      : "memory");
 }
+__device__ __forceinline__ void tmem_st_32x32b_x16_fill(uint32_t taddr, uint32_t v) {
+#pragma unroll
+    for (int c = 0; c < 16; c += 8)
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr + c),
+                     "r"(v)
+                     : "memory");
+}
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {

@@ -4,7 +4,7 @@
 // int8 under the same rotation) and the recipe (transform=fwht128 group=128
 // scale=bf16 clamp=sym).
 //
-// fwht128_quant_kernel: one warp per 128-wide block of a row.  Lane l holds
+// fwht128_warp / fwht128_quant_kernel: one warp per 128-wide block of a row.  Lane l holds
 // elements 4l .. 4l+3 in fp32.  The textbook in-place butterflies run stage
 // by stage, h = 1, 2, 4, ..., 64, each pair (a, b) at distance h becoming
 // (a + b, a - b): stages 1 and 2 inside the lane, stages 4 .. 64 between
@@ -23,17 +23,9 @@
 
 namespace w8a8 {
 
-__global__ void __launch_bounds__(256) fwht128_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
-                                                            int8_t* __restrict__ q, uint16_t* __restrict__ s) {
-    const int lane = threadIdx.x & 31;
-    const int64_t G = K / 128;
-    const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (blk >= M * G) return;
-    const int64_t m = blk / G, g = blk % G;
-    const uint16_t* src = x + m * K + g * 128 + 4 * lane;
-    const uint2 raw = *reinterpret_cast<const uint2*>(src);
-    float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u), __uint_as_float(raw.y << 16),
-                  __uint_as_float(raw.y & 0xffff0000u)};
+// The rotation of one 128-wide block by one warp: lane l holds elements
+// 4l .. 4l+3 in fp32 (see above for the stage order).
+__device__ __forceinline__ void fwht128_warp(float (&v)[4], int lane) {
     // h = 1: (0,1), (2,3)
     {
         const float a0 = v[0], b0 = v[1], a1 = v[2], b1 = v[3];
@@ -60,10 +52,16 @@ __global__ void __launch_bounds__(256) fwht128_quant_kernel(const uint16_t* __re
             v[j] = upper ? __fsub_rn(o, v[j]) : __fadd_rn(v[j], o);
         }
     }
+}
+
+// Group quantization of a rotated block held as above: the bf16 scale
+// s = bf16_rne(max |x'| / 127) (returned in sb, every lane) and this lane's
+// four codes clamp(rne(x' / float(s)), +-127), packed little-endian.
+__device__ __forceinline__ uint32_t fwht128_codes(const float (&v)[4], uint16_t& sb) {
     float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const uint16_t sb = float_to_bf16_bits(__fdiv_rn(amax, 127.0f));
+    sb = float_to_bf16_bits(__fdiv_rn(amax, 127.0f));
     const float sf = bf16_bits_to_float(sb);
     uint32_t pk = 0u;
     if (sf != 0.0f) {
@@ -71,6 +69,43 @@ __global__ void __launch_bounds__(256) fwht128_quant_kernel(const uint16_t* __re
 #pragma unroll
         for (int j = 0; j < 4; ++j) pk |= (uint32_t)(uint8_t)(int8_t)quant_code_rcp(v[j], sf, rcp) << (8 * j);
     }
+    return pk;
+}
+
+__device__ __forceinline__ void fwht128_load4(const uint16_t* src, float (&v)[4]) {
+    const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(src));
+    v[0] = __uint_as_float(raw.x << 16);
+    v[1] = __uint_as_float(raw.x & 0xffff0000u);
+    v[2] = __uint_as_float(raw.y << 16);
+    v[3] = __uint_as_float(raw.y & 0xffff0000u);
+}
+__device__ __forceinline__ void fwht128_load4(const float* src, float (&v)[4]) {
+    const float4 raw = __ldcg(reinterpret_cast<const float4*>(src));
+    v[0] = raw.x;
+    v[1] = raw.y;
+    v[2] = raw.z;
+    v[3] = raw.w;
+}
+
+// One warp per 128-wide block of a row; bf16 rows (activations, weights) or
+// fp32 rows (the routed experts' gated intermediate).  On a chain with
+// programmatic dependent launch it waits for the kernel before it (a no-op
+// otherwise) and reads its rows with coherent loads.
+template <typename Tin>
+__global__ void __launch_bounds__(256) fwht128_quant_kernel(const Tin* __restrict__ x, int64_t M, int64_t K,
+                                                            int8_t* __restrict__ q, uint16_t* __restrict__ s) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int lane = threadIdx.x & 31;
+    const int64_t G = K / 128;
+    const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (blk >= M * G) return;
+    const int64_t m = blk / G, g = blk % G;
+    float v[4];
+    fwht128_load4(x + m * K + g * 128 + 4 * lane, v);
+    fwht128_warp(v, lane);
+    uint16_t sb;
+    const uint32_t pk = fwht128_codes(v, sb);
     *reinterpret_cast<uint32_t*>(q + m * K + g * 128 + 4 * lane) = pk;
     if (lane == 0) s[m * G + g] = sb;
 }

@@ -42,22 +42,29 @@ constexpr int kMsBM = 128;          // weight rows per group (MMA M)
 constexpr int kMsBK = 128;          // bytes of K per stage
 constexpr int kMsThreads = 192;
 constexpr int kKernelIdMoeSwap = 5;
+constexpr int kMsMaxGroups = 32;    // K / 128 of the group-128 form
+constexpr int kMsSlots = 8;         // TMEM accumulators of the group-128 form: one per k block in flight
 
-template <int BN>
+template <int BN, bool G128 = false>
 struct MsSmem {
     static constexpr int kStages = BN <= 32 ? 10 : 8;
+    static constexpr int kNAcc = G128 ? kMsSlots : 2;
     static constexpr int kW = kMsBM * kMsBK;        // 16 KB
     static constexpr int kX = BN * kMsBK;           // 2 / 4 / 8 KB
     static constexpr int kStage = kW + kX;          // multiple of 1024
     static constexpr int kTiles = kStages * kStage;
-    static constexpr int kBars = (2 * kStages + 4 + 1) * 8;
+    static constexpr int kBars = (2 * kStages + 2 * kNAcc + 1) * 8;
     // the plan (tile_off, offsets, counts: 3 x 257 ints) and, per epilogue
     // buffer, the token block's row data (scale, destination, weight)
     static constexpr int kPlanOff = kTiles + kBars + 16;
     static constexpr int kPlanInts = 3 * 260;
     static constexpr int kRowOff = kPlanOff + kPlanInts * 4;
     static constexpr int kRowBytes = 2 * 3 * 64 * 4;
-    static constexpr int kBytes = 1024 + kRowOff + kRowBytes;
+    // group-128: the token block's scales, [2 buffers][group][row] fp32
+    static constexpr int kSxOff = (kRowOff + kRowBytes + 15) / 16 * 16;   // read as float4
+    static constexpr int kSxBytes = G128 ? 2 * kMsMaxGroups * BN * 4 : 0;
+    static constexpr int kBytes = 1024 + kSxOff + kSxBytes;
+    static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 struct MoeSwapArgs {
@@ -77,6 +84,9 @@ struct MoeSwapArgs {
     float* contrib;           // [T * topk, H] w * y2 at (token, slot)
     int topk;
     int early_plan;           // the plan comes two or more kernels back: read it before the wait
+    // group-128 form (K / 128 groups, bf16 scales)
+    const uint16_t* gsw;      // [E * rows, K / 128]
+    const uint16_t* gsx;      // [R, K / 128] of the sorted rows
 };
 
 // Token block b (in tile_off numbering) -> expert, first sorted row, rows;
@@ -105,20 +115,21 @@ __device__ __forceinline__ MsBlock ms_block(const int* sp, int E, int b, int BN)
 
 __device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int BN, bool GATED>
+template <int BN, bool GATED, bool G128 = false>
 __global__ void __launch_bounds__(kMsThreads, 1)
     moe_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, MoeSwapArgs a) {
     static_assert(BN == 16 || BN == 32 || BN == 64, "BN");
-    using SM = MsSmem<BN>;
+    using SM = MsSmem<BN, G128>;
     constexpr int STAGES = SM::kStages;
-    constexpr int kCols = 2 * BN >= 32 ? 2 * BN : 32;
+    constexpr int NACC = SM::kNAcc;
+    constexpr int kCols = G128 ? kMsSlots * BN : (2 * BN >= 32 ? 2 * BN : 32);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kTiles);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* mma_done = tempty + 2;
+    uint64_t* tempty = tfull + NACC;
+    uint64_t* mma_done = tempty + NACC;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -128,7 +139,7 @@ __global__ void __launch_bounds__(kMsThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NACC; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 128);
         }
@@ -210,7 +221,47 @@ __global__ void __launch_bounds__(kMsThreads, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        if (G128 && lane == 0) {
+            // one accumulator slot per k block (= group): every slot holds the
+            // conversion bias when it is released, so the MMAs always accumulate
+            // and a slot's first use waits for phase 0 like every later one
+            constexpr uint32_t idesc = idesc_i8(kMsBM, BN);
+            int stage = 0, slot = 0;
+            uint32_t phase = 0, sphase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                for (int kb = 0; kb < a.nkb; ++kb) {
+                    if (!mbar_wait_bounded(&tempty[slot], sphase, abort_flag, (kKernelIdMoeSwap << 16) | 3)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, (kKernelIdMoeSwap << 16) | 4)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(slot * BN);
+                    const uint32_t w0 = smem_u32(smem + stage * SM::kStage);
+                    const uint32_t x0 = w0 + SM::kW;
+#pragma unroll
+                    for (int kk = 0; kk < kMsBK / 32; ++kk)
+                        tc_mma_i8(d_tmem, smem_desc_k_sw128(w0 + kk * 32), smem_desc_k_sw128(x0 + kk * 32), idesc, 1u);
+                    tc_commit(&empty[stage]);
+                    tc_commit(&tfull[slot]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++slot == kMsSlots) {
+                        slot = 0;
+                        sphase ^= 1u;
+                    }
+                }
+            }
+            tc_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0u, nullptr, (kKernelIdMoeSwap << 16) | 5, 100000000ull);
+        } else if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kMsBM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
@@ -249,6 +300,145 @@ __global__ void __launch_bounds__(kMsThreads, 1)
             }
             tc_commit(mma_done);
             mbar_wait_bounded(mma_done, 0u, nullptr, (kKernelIdMoeSwap << 16) | 5, 100000000ull);
+        }
+    } else if constexpr (G128) {
+        // ---------------------------------------------------------- epilogue, group-128
+        // y[n, m] = sum over groups g ascending of fma(float(p_g), sx[m, g] * sw[n, g], y)
+        // in fp32, then * 1/128: two token rows per instruction (f32x2).  Each
+        // slot holds the bias 0x4B400000 (the bits of 1.5 * 2^23) before its
+        // MMAs, so it ends holding the float bits of 1.5 * 2^23 + p_g exactly
+        // (|p_g| <= 127^2 * 128 < 2^22) and float(p_g) is one subtraction.
+        const int quarter = warp & 3;
+        const int et = threadIdx.x - 64;   // 0 .. 127
+        float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff);   // [2][3][64]
+        float* s_sx = reinterpret_cast<float*>(smem + SM::kSxOff);     // [2][kMsMaxGroups][BN]
+        const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
+        const int G = a.nkb;
+#pragma unroll 1
+        for (int sl = 0; sl < kMsSlots; ++sl) {
+#pragma unroll
+            for (int c = 0; c < BN; c += 16) tmem_st_32x32b_x16_fill(tq + (uint32_t)(sl * BN + c), 0x4B400000u);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        for (int sl = 0; sl < kMsSlots; ++sl) mbar_arrive(&tempty[sl]);
+        // the token block's group scales: thread et holds row mm of groups
+        // g0, g0 + 128 / BN, ...; loaded one unit ahead
+        constexpr int J = BN * kMsMaxGroups / 128;
+        constexpr int kGStep = 128 / BN;
+        const int mm = et & (BN - 1), g0 = et / BN;
+        float nx_g[J];
+        float nx_w = 0.0f;
+        int nx_dst = 0;
+        auto fetch = [&](int u) {
+            const int b = u / a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            const bool have = mm < k.valid;
+            const uint16_t* src = a.gsx + (int64_t)(k.row0 + mm) * G;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int gg = g0 + kGStep * j;
+                nx_g[j] = (have && gg < G) ? bf16_bits_to_float(__ldcg(src + gg)) : 0.0f;
+            }
+            if constexpr (!GATED) {
+                if (et < k.valid) {
+                    const int r = k.row0 + et;
+                    nx_dst = __ldcg(a.row_tok + r) * a.topk + __ldcg(a.row_slot + r);
+                    nx_w = __ldcg(a.row_w + r);
+                }
+            }
+        };
+        if ((int)blockIdx.x < nunits) fetch(blockIdx.x);
+        int slot = 0, buf = 0;
+        uint32_t sphase = 0;
+        const uint64_t magic2 = 0x4B4000004B400000ull;
+        const uint64_t inv2 = f2_pack(0.0078125f, 0.0078125f);
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+            const int b = u / a.ngroups, g = u - b * a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            float* rs = s_row + buf * 3 * 64;
+            float* sxs = s_sx + buf * kMsMaxGroups * BN;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int gg = g0 + kGStep * j;
+                if (gg < G) sxs[gg * BN + mm] = nx_g[j];
+            }
+            if constexpr (!GATED) {
+                if (et < BN) {
+                    const bool have = et < k.valid;
+                    rs[64 + et] = __int_as_float(have ? nx_dst : 0);
+                    rs[128 + et] = have ? nx_w : 0.0f;
+                }
+            }
+            if (u + (int)gridDim.x < nunits) fetch(u + gridDim.x);
+            ms_epi_sync();   // also: every warp is done with this buffer's use two units ago
+            buf ^= 1;
+            const int n = g * kMsBM + quarter * 32 + lane;   // weight row of expert e
+            const uint16_t* swrow = a.gsw + ((int64_t)k.e * a.rows + n) * G;
+            float sw_next = bf16_bits_to_float(__ldg(swrow));
+            uint64_t y2[BN / 2];
+#pragma unroll
+            for (int i = 0; i < BN / 2; ++i) y2[i] = 0ull;
+            bool ok = true;
+            for (int kb = 0; kb < G; ++kb) {
+                const float swg = sw_next;
+                if (kb + 1 < G) sw_next = bf16_bits_to_float(__ldg(swrow + kb + 1));
+                if (!mbar_wait_bounded(&tfull[slot], sphase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t sw2 = f2_pack(swg, swg);
+                const float* sxk = sxs + kb * BN;
+#pragma unroll
+                for (int c = 0; c < BN; c += 16) {
+                    const uint32_t ta = tq + (uint32_t)(slot * BN + c);
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(ta, r);
+                    tc_wait_ld();
+                    tmem_st_32x32b_x16_fill(ta, 0x4B400000u);
+                    if (c + 16 == BN) {   // the slot goes back to the MMA
+                        tc_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&tempty[slot]);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 s4 = *reinterpret_cast<const float4*>(sxk + c + 4 * q);
+                        const uint64_t sc01 = f2_mul(f2_pack(s4.x, s4.y), sw2);
+                        const uint64_t sc23 = f2_mul(f2_pack(s4.z, s4.w), sw2);
+                        const uint64_t p01 =
+                            f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
+                        const uint64_t p23 =
+                            f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
+                        y2[c / 2 + 2 * q] = f2_fma(p01, sc01, y2[c / 2 + 2 * q]);
+                        y2[c / 2 + 2 * q + 1] = f2_fma(p23, sc23, y2[c / 2 + 2 * q + 1]);
+                    }
+                }
+                if (++slot == kMsSlots) {
+                    slot = 0;
+                    sphase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            float v[BN];
+#pragma unroll
+            for (int i = 0; i < BN / 2; ++i) f2_unpack(f2_mul(y2[i], inv2), v[2 * i], v[2 * i + 1]);
+            if constexpr (GATED) {
+                const int I = a.rows >> 1;
+                float* arow = a.a_out + (int64_t)k.row0 * I + (n >> 1);
+#pragma unroll
+                for (int m = 0; m < BN; ++m) {
+                    const float up = __shfl_xor_sync(0xffffffffu, v[m], 1);   // row n + 1 (odd lane)
+                    if (m < k.valid && !(lane & 1)) arow[(int64_t)m * I] = __fmul_rn(silu_proj(v[m]), up);
+                }
+            } else {
+                const int H = a.rows;
+#pragma unroll
+                for (int m = 0; m < BN; ++m)
+                    if (m < k.valid)
+                        a.contrib[(int64_t)__float_as_int(rs[64 + m]) * H + n] = __fmul_rn(rs[128 + m], v[m]);
+            }
         }
     } else {
         // ---------------------------------------------------------- epilogue

@@ -16,6 +16,7 @@
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
 #include "moe.cuh"
+#include "moe_g128.cuh"
 #include "moe_swap.cuh"
 #include "quant.cuh"
 #include "w8a8.h"
@@ -515,10 +516,10 @@ int launch_tc_grouped(const int8_t* A, int64_t rowsA, const int8_t* B, int E, Tc
 
 // Swap-AB expert GEMM over token blocks of BN rows: W = an expert stack
 // viewed as [E * rows, K], X = the sorted codes [R, K].
-template <int BN, bool GATED>
+template <int BN, bool GATED, bool G128 = false>
 int launch_moe_swap(const int8_t* W, const int8_t* X, int64_t R, MoeSwapArgs a, int64_t nb_max, cudaStream_t st) {
-    using SM = MsSmem<BN>;
-    auto kern = moe_swap_kernel<BN, GATED>;
+    using SM = MsSmem<BN, G128>;
+    auto kern = moe_swap_kernel<BN, GATED, G128>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
@@ -980,6 +981,159 @@ int w8a8_mlp_forward(const uint16_t* x, const int8_t* w13, const float* s13, con
             return W8A8_ERR_CUDA;
         if (dbg->sa && cudaMemcpyAsync(dbg->sa, w.sa, (size_t)M * 4, cudaMemcpyDeviceToDevice, st))
             return W8A8_ERR_CUDA;
+    }
+    return W8A8_OK;
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------- MoE, FWHT128 grid
+namespace {
+struct MoeG128Ws {
+    int32_t* ids;
+    float* wts;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* active;
+    int32_t* n_active;
+    int32_t* tile_off;
+    int32_t* rank;
+    int32_t* done;
+    int32_t* row_of;
+    int32_t* row_tok;
+    int32_t* row_slot;
+    float* row_w;
+    int8_t* xq;       // [R, H] rotated codes of x, expert-sorted rows
+    uint16_t* sxg;    // [R, H / 128]
+    float* a;         // [R, I] fp32 gated intermediate
+    int8_t* qa;       // [R, I] its rotated codes
+    uint16_t* sag;    // [R, I / 128]
+    float* out;       // [R, H] w * y2 at (token, slot)
+    size_t bytes;
+};
+
+MoeG128Ws moe_g128_carve(void* base, int64_t T, int E, int H, int I, int topk) {
+    MoeG128Ws w;
+    const int64_t R = T * topk;
+    uint8_t* p = reinterpret_cast<uint8_t*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* r = p ? p + o : nullptr;
+        o += align_up(bytes, 256);
+        return r;
+    };
+    w.ids = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.wts = reinterpret_cast<float*>(take((size_t)R * 4));
+    w.counts = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));   // counts and the plan's CTA counter
+    w.done = w.counts + E;
+    w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+    w.active = reinterpret_cast<int32_t*>(take((size_t)E * 4));
+    w.n_active = reinterpret_cast<int32_t*>(take(4));
+    w.tile_off = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+    w.rank = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_of = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_tok = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_slot = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    w.row_w = reinterpret_cast<float*>(take((size_t)R * 4));
+    w.xq = reinterpret_cast<int8_t*>(take((size_t)R * H));
+    w.sxg = reinterpret_cast<uint16_t*>(take((size_t)R * (H / 128) * 2));
+    w.a = reinterpret_cast<float*>(take((size_t)R * I * 4));
+    w.qa = reinterpret_cast<int8_t*>(take((size_t)R * I));
+    w.sag = reinterpret_cast<uint16_t*>(take((size_t)R * (I / 128) * 2));
+    w.out = reinterpret_cast<float*>(take((size_t)R * H * 4));
+    w.bytes = o;
+    return w;
+}
+}  // namespace
+
+extern "C" {
+
+size_t w8a8_moe_g128_workspace_size(int64_t T, int E, int H, int I, int topk) {
+    if (T <= 0 || E <= 0 || H < 128 || I < 128 || topk <= 0) return 0;
+    return moe_g128_carve(nullptr, T, E, H, I, topk).bytes;
+}
+
+int w8a8_moe_g128_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w13, const uint16_t* s13,
+                          const int8_t* w2, const uint16_t* s2, uint16_t* y, int64_t T, int E, int H, int I, int topk,
+                          void* ws, size_t ws_bytes, const w8a8_moe_g128_debug* dbg, void* stream) {
+    if (!x || !logits || !w13 || !s13 || !w2 || !s2 || !y || !ws) return W8A8_ERR_INVALID_ARG;
+    if (T <= 0 || E <= 0 || H <= 0 || I <= 0 || topk <= 0 || topk > E || topk > kMoeMaxTopk) return W8A8_ERR_INVALID_ARG;
+    if (E > 256) return W8A8_ERR_UNSUPPORTED;
+    if (H % 128 != 0 || I % 128 != 0 || H > 128 * kMoeG128MaxGroupsH || I > 2048) return W8A8_ERR_UNSUPPORTED;
+    if (T * topk > (int64_t)1 << 30 || T > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(logits, 2) || !aligned(w13, 16) || !aligned(s13, 2) || !aligned(w2, 16) ||
+        !aligned(s2, 2) || !aligned(y, 16) || !aligned(ws, 256))
+        return W8A8_ERR_INVALID_ARG;
+    if (ws_bytes < w8a8_moe_g128_workspace_size(T, E, H, I, topk)) return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    MoeG128Ws w = moe_g128_carve(ws, T, E, H, I, topk);
+    const int64_t R = T * topk;
+    int rc;
+
+    // token blocks of 16 / 32 / 64 expert-sorted rows, by the average rows per expert
+    const int64_t avg_rows = (R + E - 1) / E;
+    const int bn = avg_rows <= 12 ? 16 : (avg_rows <= 24 ? 32 : 64);
+    MoePlan plan = {w.counts, w.offsets, w.active, w.n_active, w.tile_off, w.rank, w.done, bn};
+    MoeRows rows = {w.ids, w.wts, w.rank, w.offsets, w.row_of, w.row_tok, w.row_slot, w.row_w};
+    if (cudaMemsetAsync(w.counts, 0, (size_t)(E + 1) * 4, st) != cudaSuccess) return W8A8_ERR_CUDA;
+    moe_route_plan_kernel<8><<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits, T, E, topk, w.ids, w.wts, plan);
+    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+    rc = launch_chained(moe_fwht_scatter_kernel, (unsigned)T, (unsigned)(32 * (H / 128)), st, x, H, topk, rows, w.xq,
+                        w.sxg, dbg ? dbg->qx : (int8_t*)nullptr, dbg ? dbg->sx : (uint16_t*)nullptr);
+    if (rc != W8A8_OK) return rc;
+
+    const int64_t nb_max = moe_max_blocks(R, E, bn);
+    MoeSwapArgs a1 = {};
+    a1.counts = w.counts;
+    a1.offsets = w.offsets;
+    a1.tile_off = w.tile_off;
+    a1.E = E;
+    a1.rows = 2 * I;
+    a1.K = H;
+    a1.ngroups = (2 * I) / 128;
+    a1.nkb = H / 128;
+    a1.a_out = w.a;
+    a1.early_plan = 1;   // the plan comes two kernels back
+    a1.gsw = s13;
+    a1.gsx = w.sxg;
+    MoeSwapArgs a2 = a1;
+    a2.rows = H;
+    a2.K = I;
+    a2.ngroups = H / 128;
+    a2.nkb = I / 128;
+    a2.gsw = s2;
+    a2.gsx = w.sag;
+    a2.row_tok = w.row_tok;
+    a2.row_slot = w.row_slot;
+    a2.row_w = w.row_w;
+    a2.contrib = w.out;
+    a2.topk = topk;
+    rc = bn == 16 ? launch_moe_swap<16, true, true>(w13, w.xq, R, a1, nb_max, st)
+       : bn == 32 ? launch_moe_swap<32, true, true>(w13, w.xq, R, a1, nb_max, st)
+                  : launch_moe_swap<64, true, true>(w13, w.xq, R, a1, nb_max, st);
+    if (rc != W8A8_OK) return rc;
+    // the intermediate rotated along I and group-quantized
+    const int64_t blocks = R * (I / 128);
+    rc = launch_chained(fwht128_quant_kernel<float>, (unsigned)((blocks + 7) / 8), 256u, st, (const float*)w.a, R,
+                        (int64_t)I, w.qa, w.sag);
+    if (rc != W8A8_OK) return rc;
+    rc = bn == 16 ? launch_moe_swap<16, false, true>(w2, w.qa, R, a2, nb_max, st)
+       : bn == 32 ? launch_moe_swap<32, false, true>(w2, w.qa, R, a2, nb_max, st)
+                  : launch_moe_swap<64, false, true>(w2, w.qa, R, a2, nb_max, st);
+    if (rc != W8A8_OK) return rc;
+    rc = launch_chained(moe_finalize_kernel, (unsigned)((T * H / 4 + 255) / 256), 256u, st, (const float*)w.out, y, T,
+                        H, topk);
+    if (rc != W8A8_OK) return rc;
+    if (!dbg) return W8A8_OK;
+    if (dbg->topk_ids && cudaMemcpyAsync(dbg->topk_ids, w.ids, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
+        return W8A8_ERR_CUDA;
+    if (dbg->topk_w && cudaMemcpyAsync(dbg->topk_w, w.wts, (size_t)R * 4, cudaMemcpyDeviceToDevice, st))
+        return W8A8_ERR_CUDA;
+    if (dbg->counts && cudaMemcpyAsync(dbg->counts, w.counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, st))
+        return W8A8_ERR_CUDA;
+    if (dbg->qa || dbg->sa) {
+        moe_debug_gather_g128_kernel<<<(unsigned)R, 128, 0, st>>>(w.qa, w.sag, w.row_of, R, I, dbg->qa, dbg->sa);
+        return last_launch_status();
     }
     return W8A8_OK;
 }

@@ -24,7 +24,7 @@ EXPORTS = (
     "w8a8_quant_act", "w8a8_quant_rows_f32", "w8a8_linear_workspace_size", "w8a8_linear",
     "w8a8_linear_noalloc_scratch_size", "w8a8_linear_noalloc",
     "w8a8_gemm_workspace_size", "w8a8_gemm_q", "w8a8_gemm_s32", "w8a8_moe_workspace_size",
-    "w8a8_moe_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
+    "w8a8_moe_forward", "w8a8_moe_g128_workspace_size", "w8a8_moe_g128_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
     "w8a8_exp_proj",
     "w8a8_get_device_error", "w8a8_debug_wait_timeout", "w8a8_status_str", "w8a8_version",
 )
@@ -36,6 +36,12 @@ class W8A8Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+class MoeG128Debug(ctypes.Structure):
+    _fields_ = [("topk_ids", ctypes.c_void_p), ("topk_w", ctypes.c_void_p), ("counts", ctypes.c_void_p),
+                ("qx", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("qa", ctypes.c_void_p),
+                ("sa", ctypes.c_void_p)]
 
 
 class MlpDebug(ctypes.Structure):
@@ -70,6 +76,9 @@ def lib() -> ctypes.CDLL:
         "w8a8_moe_workspace_size": ([i64, i32, i32, i32, i32], sz),
         "w8a8_moe_forward": ([vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, sz,
                               ctypes.POINTER(MoeDebug), vp], i32),
+        "w8a8_moe_g128_workspace_size": ([i64, i32, i32, i32, i32], sz),
+        "w8a8_moe_g128_forward": ([vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, sz,
+                                   ctypes.POINTER(MoeG128Debug), vp], i32),
         "w8a8_mlp_workspace_size": ([i64, i64, i64], sz),
         "w8a8_mlp_forward": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, ctypes.POINTER(MlpDebug), vp], i32),
         "fwht128_quant": ([vp, i64, i64, vp, vp, vp], i32),
@@ -273,6 +282,49 @@ def moe_forward(x, logits, w13, s13, w2, s2, topk: int = 8, y=None, ws=None, deb
     _check(lib().w8a8_moe_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13), _ptr(w2), _ptr(s2), _ptr(y),
                                   T, E, H, I, topk, _ptr(ws), ws.numel(), dbg_p, _stream(stream)),
            "w8a8_moe_forward")
+    return (y, dbg_t) if debug else y
+
+
+# ------------------------------------------------------------------ MoE on the FWHT128 grid
+
+def moe_g128_workspace_size(T: int, E: int, H: int, I: int, topk: int) -> int:
+    return int(lib().w8a8_moe_g128_workspace_size(T, E, H, I, topk))
+
+
+def moe_g128_forward(x, logits, w13, s13, w2, s2, topk: int = 8, y=None, ws=None, debug: bool = False,
+                     stream=None):
+    """Routed experts on the FWHT128 grid: bf16 x [T,H] (unrotated), bf16 logits [T,E];
+    w13 int8 [E,2I,H] with bf16 group scales s13 [E,2I,H/128]; w2 int8 [E,H,I] with
+    s2 [E,H,I/128] (rows rotated along K and group-quantized, e.g. by fwht128_quant).
+    Returns y bf16 [T,H], or (y, debug dict) when debug."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(logits, torch.bfloat16, "logits", 2)
+    _need(w13, torch.int8, "w13", 3)
+    _need(w2, torch.int8, "w2", 3)
+    _need(s13, torch.bfloat16, "s13", 3)
+    _need(s2, torch.bfloat16, "s2", 3)
+    T, H = x.shape
+    E, I2, _ = w13.shape
+    I = I2 // 2
+    dev = x.device
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = _workspace(moe_g128_workspace_size(T, E, H, I, topk), dev)
+    dbg_t = None
+    dbg_p = None
+    if debug:
+        dbg_t = dict(topk_ids=torch.empty((T, topk), dtype=torch.int32, device=dev),
+                     topk_w=torch.empty((T, topk), dtype=torch.float32, device=dev),
+                     counts=torch.empty(E, dtype=torch.int32, device=dev),
+                     qx=torch.empty((T, H), dtype=torch.int8, device=dev),
+                     sx=torch.empty((T, H // 128), dtype=torch.bfloat16, device=dev),
+                     qa=torch.empty((T, topk, I), dtype=torch.int8, device=dev),
+                     sa=torch.empty((T, topk, I // 128), dtype=torch.bfloat16, device=dev))
+        dbg_p = ctypes.pointer(MoeG128Debug(*[v.data_ptr() for v in dbg_t.values()]))
+    _check(lib().w8a8_moe_g128_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13), _ptr(w2), _ptr(s2), _ptr(y),
+                                       T, E, H, I, topk, _ptr(ws), ws.numel(), dbg_p, _stream(stream)),
+           "w8a8_moe_g128_forward")
     return (y, dbg_t) if debug else y
 
 
