@@ -169,6 +169,16 @@ __device__ __forceinline__ void tmem_st_32x32b_x32_fill(uint32_t taddr, uint32_t
                      "r"(v)
                      : "memory");
 }
+__device__ __forceinline__ void tmem_st_32x32b_x8_fill(uint32_t taddr, uint32_t v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr), "r"(v)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_st_32x32b_x16_fill(uint32_t taddr, uint32_t v) {
 #pragma unroll
     for (int c = 0; c < 16; c += 8)
@@ -250,7 +260,10 @@ __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
 __device__ __forceinline__ float exp_proj(float x) {
     x = fminf(fmaxf(x, -87.0f), 88.0f);
     const float t = __fmul_rn(x, 1.44269502162933349609375f);
-    const float n = rintf(t);
+    // n = rne(t) through the 1.5 * 2^23 bias (|t| <= 127): tb holds it in its
+    // low mantissa bits, so both n and its integer come without a conversion
+    const float tb = __fadd_rn(t, 12582912.0f);
+    const float n = __fsub_rn(tb, 12582912.0f);
     float r = __fmaf_rn(-n, 0.693359375f, x);
     r = __fmaf_rn(-n, -2.12194440e-4f, r);
     float p = 1.0f / 5040.0f;
@@ -261,7 +274,7 @@ __device__ __forceinline__ float exp_proj(float x) {
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
-    const int ni = __float2int_rn(n);
+    const int ni = (int)(__float_as_uint(tb) - 0x4B400000u);
     return __fmul_rn(p, __int_as_float((ni + 127) << 23));
 }
 

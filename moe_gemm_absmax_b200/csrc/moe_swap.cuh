@@ -29,8 +29,9 @@
 // the weight tiles of its first stages before it waits for the codes of the
 // kernel just before.
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-// warps 2..5 epilogue (TMEM lane quarters).  All waits are bounded.
+// Roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..5
+// epilogue (TMEM lane quarters); the group-128 form has 8 epilogue warps
+// (lane quarter x half of the token block's columns).  All waits are bounded.
 #pragma once
 
 #include "common.cuh"
@@ -40,7 +41,6 @@ namespace w8a8 {
 
 constexpr int kMsBM = 128;          // weight rows per group (MMA M)
 constexpr int kMsBK = 128;          // bytes of K per stage
-constexpr int kMsThreads = 192;
 constexpr int kKernelIdMoeSwap = 5;
 constexpr int kMsMaxGroups = 32;    // K / 128 of the group-128 form
 constexpr int kMsSlots = 8;         // TMEM accumulators of the group-128 form: one per k block in flight
@@ -113,10 +113,15 @@ __device__ __forceinline__ MsBlock ms_block(const int* sp, int E, int b, int BN)
     return k;
 }
 
-__device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+template <int NT>
+__device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+
+// Threads: producer warp, MMA warp, then 4 epilogue warps (8 for the group-128 form).
+template <bool G128>
+constexpr int ms_threads() { return G128 ? 320 : 192; }
 
 template <int BN, bool GATED, bool G128 = false>
-__global__ void __launch_bounds__(kMsThreads, 1)
+__global__ void __launch_bounds__(ms_threads<G128>(), 1)
     moe_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, MoeSwapArgs a) {
     static_assert(BN == 16 || BN == 32 || BN == 64, "BN");
     using SM = MsSmem<BN, G128>;
@@ -141,7 +146,7 @@ __global__ void __launch_bounds__(kMsThreads, 1)
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], G128 ? 256 : 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -308,24 +313,27 @@ __global__ void __launch_bounds__(kMsThreads, 1)
         // slot holds the bias 0x4B400000 (the bits of 1.5 * 2^23) before its
         // MMAs, so it ends holding the float bits of 1.5 * 2^23 + p_g exactly
         // (|p_g| <= 127^2 * 128 < 2^22) and float(p_g) is one subtraction.
+        // Eight warps: TMEM lane quarter (warp % 4) x half of the block's columns.
+        constexpr int HC = BN / 2;
         const int quarter = warp & 3;
-        const int et = threadIdx.x - 64;   // 0 .. 127
+        const int c0 = ((warp - 2) >> 2) * HC;
+        const int et = threadIdx.x - 64;   // 0 .. 255
         float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff);   // [2][3][64]
         float* s_sx = reinterpret_cast<float*>(smem + SM::kSxOff);     // [2][kMsMaxGroups][BN]
-        const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0;
         const int G = a.nkb;
 #pragma unroll 1
         for (int sl = 0; sl < kMsSlots; ++sl) {
 #pragma unroll
-            for (int c = 0; c < BN; c += 16) tmem_st_32x32b_x16_fill(tq + (uint32_t)(sl * BN + c), 0x4B400000u);
+            for (int c = 0; c < HC; c += 8) tmem_st_32x32b_x8_fill(tq + (uint32_t)(sl * BN + c), 0x4B400000u);
         }
         tc_wait_st();
         tc_fence_before();
         for (int sl = 0; sl < kMsSlots; ++sl) mbar_arrive(&tempty[sl]);
         // the token block's group scales: thread et holds row mm of groups
-        // g0, g0 + 128 / BN, ...; loaded one unit ahead
-        constexpr int J = BN * kMsMaxGroups / 128;
-        constexpr int kGStep = 128 / BN;
+        // g0, g0 + 256 / BN, ...; loaded one unit ahead
+        constexpr int J = BN * kMsMaxGroups / 256;
+        constexpr int kGStep = 256 / BN;
         const int mm = et & (BN - 1), g0 = et / BN;
         float nx_g[J];
         float nx_w = 0.0f;
@@ -371,14 +379,14 @@ __global__ void __launch_bounds__(kMsThreads, 1)
                 }
             }
             if (u + (int)gridDim.x < nunits) fetch(u + gridDim.x);
-            ms_epi_sync();   // also: every warp is done with this buffer's use two units ago
+            ms_epi_sync<256>();   // also: every warp is done with this buffer's use two units ago
             buf ^= 1;
             const int n = g * kMsBM + quarter * 32 + lane;   // weight row of expert e
             const uint16_t* swrow = a.gsw + ((int64_t)k.e * a.rows + n) * G;
             float sw_next = bf16_bits_to_float(__ldg(swrow));
-            uint64_t y2[BN / 2];
+            uint64_t y2[HC / 2];
 #pragma unroll
-            for (int i = 0; i < BN / 2; ++i) y2[i] = 0ull;
+            for (int i = 0; i < HC / 2; ++i) y2[i] = 0ull;
             bool ok = true;
             for (int kb = 0; kb < G; ++kb) {
                 const float swg = sw_next;
@@ -389,55 +397,60 @@ __global__ void __launch_bounds__(kMsThreads, 1)
                 }
                 tc_fence_after();
                 const uint64_t sw2 = f2_pack(swg, swg);
-                const float* sxk = sxs + kb * BN;
+                const float* sxk = sxs + kb * BN + c0;
+                // this warp's columns into registers (one wait), the bias back
+                // into TMEM, the promotion while those stores land, the release
+                const uint32_t ta = tq + (uint32_t)(slot * BN);
+                uint32_t r[HC];
+                if constexpr (HC == 8) tmem_ld_32x32b_x8(ta, r);
+                else if constexpr (HC == 16) tmem_ld_32x32b_x16(ta, r);
+                else tmem_ld_32x32b_x32(ta, r);
+                tc_wait_ld();
 #pragma unroll
-                for (int c = 0; c < BN; c += 16) {
-                    const uint32_t ta = tq + (uint32_t)(slot * BN + c);
-                    uint32_t r[16];
-                    tmem_ld_32x32b_x16(ta, r);
-                    tc_wait_ld();
-                    tmem_st_32x32b_x16_fill(ta, 0x4B400000u);
-                    if (c + 16 == BN) {   // the slot goes back to the MMA
-                        tc_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(&tempty[slot]);
-                    }
+                for (int c = 0; c < HC; c += 8) tmem_st_32x32b_x8_fill(ta + (uint32_t)c, 0x4B400000u);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 s4 = *reinterpret_cast<const float4*>(sxk + c + 4 * q);
-                        const uint64_t sc01 = f2_mul(f2_pack(s4.x, s4.y), sw2);
-                        const uint64_t sc23 = f2_mul(f2_pack(s4.z, s4.w), sw2);
-                        const uint64_t p01 =
-                            f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
-                        const uint64_t p23 =
-                            f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
-                        y2[c / 2 + 2 * q] = f2_fma(p01, sc01, y2[c / 2 + 2 * q]);
-                        y2[c / 2 + 2 * q + 1] = f2_fma(p23, sc23, y2[c / 2 + 2 * q + 1]);
-                    }
+                for (int q = 0; q < HC / 4; ++q) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(sxk + 4 * q);
+                    const uint64_t sc01 = f2_mul(f2_pack(s4.x, s4.y), sw2);
+                    const uint64_t sc23 = f2_mul(f2_pack(s4.z, s4.w), sw2);
+                    const uint64_t p01 = f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
+                    const uint64_t p23 =
+                        f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
+                    y2[2 * q] = f2_fma(p01, sc01, y2[2 * q]);
+                    y2[2 * q + 1] = f2_fma(p23, sc23, y2[2 * q + 1]);
                 }
+                tc_wait_st();
+                tc_fence_before();
+                mbar_arrive(&tempty[slot]);   // the slot goes back to the MMA
                 if (++slot == kMsSlots) {
                     slot = 0;
                     sphase ^= 1u;
                 }
             }
             if (!ok) break;
-            float v[BN];
+            float v[HC];
 #pragma unroll
-            for (int i = 0; i < BN / 2; ++i) f2_unpack(f2_mul(y2[i], inv2), v[2 * i], v[2 * i + 1]);
+            for (int i = 0; i < HC / 2; ++i) f2_unpack(f2_mul(y2[i], inv2), v[2 * i], v[2 * i + 1]);
             if constexpr (GATED) {
+                // lanes 2i (gate_i) and 2i+1 (up_i) split the columns: the even
+                // lane finishes the first half, the odd lane the second
                 const int I = a.rows >> 1;
                 float* arow = a.a_out + (int64_t)k.row0 * I + (n >> 1);
+                const bool odd = lane & 1;
 #pragma unroll
-                for (int m = 0; m < BN; ++m) {
-                    const float up = __shfl_xor_sync(0xffffffffu, v[m], 1);   // row n + 1 (odd lane)
-                    if (m < k.valid && !(lane & 1)) arow[(int64_t)m * I] = __fmul_rn(silu_proj(v[m]), up);
+                for (int j = 0; j < HC / 2; ++j) {
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? v[j] : v[j + HC / 2], 1);
+                    const float gv = odd ? other : v[j];
+                    const float uv = odd ? v[j + HC / 2] : other;
+                    const int m = c0 + j + (odd ? HC / 2 : 0);
+                    if (m < k.valid) arow[(int64_t)m * I] = __fmul_rn(silu_proj(gv), uv);
                 }
             } else {
                 const int H = a.rows;
 #pragma unroll
-                for (int m = 0; m < BN; ++m)
-                    if (m < k.valid)
-                        a.contrib[(int64_t)__float_as_int(rs[64 + m]) * H + n] = __fmul_rn(rs[128 + m], v[m]);
+                for (int m = 0; m < HC; ++m)
+                    if (c0 + m < k.valid)
+                        a.contrib[(int64_t)__float_as_int(rs[64 + c0 + m]) * H + n] = __fmul_rn(rs[128 + c0 + m], v[m]);
             }
         }
     } else {
@@ -477,7 +490,7 @@ __global__ void __launch_bounds__(kMsThreads, 1)
                 }
                 if (u + (int)gridDim.x < nunits) fetch(u + gridDim.x);
             }
-            ms_epi_sync();   // also: every warp is done with this buffer's use two units ago
+            ms_epi_sync<128>();   // also: every warp is done with this buffer's use two units ago
             buf ^= 1;
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) break;
             tc_fence_after();

@@ -536,7 +536,7 @@ int launch_moe_swap(const int8_t* W, const int8_t* X, int64_t R, MoeSwapArgs a, 
     const int sms = device_sms(dev);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units < sms ? units : sms), 1, 1);
-    cfg.blockDim = dim3(kMsThreads, 1, 1);
+    cfg.blockDim = dim3(ms_threads<G128>(), 1, 1);
     cfg.dynamicSmemBytes = SM::kBytes;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
