@@ -81,6 +81,8 @@ def lib():
             L.oracle_fwht128_quant.argtypes = [vp, i64, i64, vp, vp, vp]
             L.oracle_gemm_g128.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             L.oracle_fwht128_quant_f32.argtypes = [vp, i64, i64, vp, vp]
+            L.oracle_group128_quant.argtypes = [vp, i64, i64, vp, vp]
+            L.oracle_gemm_group128.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             L.oracle_moe_g128_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32,
                                                   vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.oracle_set_threads.argtypes = [i32]
@@ -338,6 +340,30 @@ def gemm_g128(qx, sx_bits, qw, sw_bits):
     y = np.empty((M, N), np.uint16)
     y32 = np.empty((M, N), np.float32)
     lib().oracle_gemm_g128(_p(qx), _p(sx), _p(qw), _p(sw), M, N, K, _p(y), _p(y32))
+    return y, y32
+
+
+def group128_quant(x_bits):
+    """Group-128 quant without the rotation (the head's grid): returns
+    (codes int8 [M,K], scales bf16 bits [M,K/128])."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    assert K % 128 == 0
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M, K // 128), np.uint16)
+    lib().oracle_group128_quant(_p(x), M, K, _p(q), _p(s))
+    return q, s
+
+
+def gemm_group128(qx, sx_bits, qw, sw_bits):
+    """Group-128 GEMM on the unrotated grid (no 1/128): returns (y bf16 bits, y fp32)."""
+    qx, qw = _c(qx, np.int8), _c(qw, np.int8)
+    sx, sw = _c(sx_bits, np.uint16), _c(sw_bits, np.uint16)
+    M, K = qx.shape
+    N = qw.shape[0]
+    y = np.empty((M, N), np.uint16)
+    y32 = np.empty((M, N), np.float32)
+    lib().oracle_gemm_group128(_p(qx), _p(sx), _p(qw), _p(sw), M, N, K, _p(y), _p(y32))
     return y, y32
 
 

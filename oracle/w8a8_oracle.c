@@ -532,14 +532,45 @@ void oracle_fwht128_quant_f32(const float* x, int64_t M, int64_t K, int8_t* q, b
 }
 
 /* ------------------------------------------------------------------ */
-/* a13: group-128 scaled GEMM in the rotated domain.                    */
+/* Group-128 quantization without the rotation (f3: [IQ8R] file table,  */
+/* Head: "the lm_head int8 with a bf16 scale per row and 128"; recipe    */
+/* row output.weight: codes=i8 group=128 scale=bf16 clamp=sym, no        */
+/* transform).  Each 128-wide block of each row: s = bf16_rne(absmax /  */
+/* 127), codes from that stored scale -- the block quantizer above       */
+/* without the butterflies.                                              */
+/* ------------------------------------------------------------------ */
+void oracle_group128_quant(const bf16_t* x, int64_t M, int64_t K, int8_t* q, bf16_t* s)
+{
+    int64_t G = K / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < G; ++g) {
+            float v[128];
+            for (int k = 0; k < 128; ++k) v[k] = oracle_bf16_to_f32(x[m * K + g * 128 + k]);
+            float amax = 0.0f;
+            for (int k = 0; k < 128; ++k) { float a = fabsf(v[k]); if (a > amax) amax = a; }
+            bf16_t sb = oracle_f32_to_bf16(amax / 127.0f);
+            float sf = oracle_bf16_to_f32(sb);
+            s[m * G + g] = sb;
+            for (int k = 0; k < 128; ++k) {
+                int8_t code = 0;
+                if (sf != 0.0f) code = clamp_sym127(rne_to_int(v[k] / sf));
+                q[m * K + g * 128 + k] = code;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* a13: group-128 scaled GEMM.                                          */
 /*   p_g = sum_{k in group g} qx[m,k] qw[n,k]            (int32, exact)   */
 /*   acc = fma(float(p_g), float(sx[m,g]) * float(sw[n,g]), acc), g asc  */
-/*   y = bf16_rne(acc * (1/128))                                          */
-/* 1/128 undoes H H^T = 128 I of the unnormalised rotation.              */
+/*   y = bf16_rne(acc * post)                                             */
+/* post = 1/128 in the rotated domain (it undoes H H^T = 128 I of the    */
+/* unnormalised rotation), 1 on the unrotated grid of the head (f3).     */
 /* ------------------------------------------------------------------ */
-void oracle_gemm_g128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, const bf16_t* sw,
-                      int64_t M, int64_t N, int64_t K, bf16_t* y, float* y32)
+static void gemm_group_scaled(const int8_t* qx, const bf16_t* sx, const int8_t* qw, const bf16_t* sw,
+                              int64_t M, int64_t N, int64_t K, float post, bf16_t* y, float* y32)
 {
     int64_t G = K / 128;
     #pragma omp parallel for schedule(static)
@@ -553,11 +584,23 @@ void oracle_gemm_g128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, cons
                 float sc = oracle_bf16_to_f32(sx[m * G + g]) * oracle_bf16_to_f32(sw[n * G + g]);
                 acc = fmaf((float)p, sc, acc);
             }
-            float r = acc * 0.0078125f;
+            float r = acc * post;
             if (y) y[m * N + n] = oracle_f32_to_bf16(r);
             if (y32) y32[m * N + n] = r;
         }
     }
+}
+
+void oracle_gemm_g128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, const bf16_t* sw,
+                      int64_t M, int64_t N, int64_t K, bf16_t* y, float* y32)
+{
+    gemm_group_scaled(qx, sx, qw, sw, M, N, K, 0.0078125f, y, y32);
+}
+
+void oracle_gemm_group128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, const bf16_t* sw,
+                          int64_t M, int64_t N, int64_t K, bf16_t* y, float* y32)
+{
+    gemm_group_scaled(qx, sx, qw, sw, M, N, K, 1.0f, y, y32);
 }
 
 /* ------------------------------------------------------------------ */
