@@ -552,13 +552,39 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         else:
             rec["roofline"] = {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"}
         out[f"hadamard_M{M}"] = rec
+    # ---- head-shaped group-128 GEMM on the unrotated grid (N = 131072 rows, K = 2048)
+    del qw, sw
+    HN, HK = HEAD["N"], HEAD["K"]
+    hw = torch.randn(HN, HK, generator=torch.Generator(device=dev).manual_seed(5), device=dev) * 0.02
+    qw, sw = w8a8.group128_quant(hw.to(torch.bfloat16))
+    del hw
+    for M in (1, 8):
+        xb, _ = inputs.hadamard_linear(M, M, K=HK, N=16)
+        x = bf16_dev(torch, xb, dev)
+        y = torch.empty((M, HN), dtype=torch.bfloat16, device=dev)
+
+        def fn():
+            q, s = w8a8.group128_quant(x)
+            w8a8.linear_group128(q, s, qw, sw, y=y)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        byts = HN * HK + 2 * HN * (HK // 128) + 2 * M * HK + 2 * M * HN
+        gbs = byts / (t * 1e-3) / 1e9
+        out[f"head_group128_M{M}"] = {"ms": t, "gbs": gbs, "roofline": {"bound": "hbm", "frac": gbs / hbm, "peak": hbm,
+                                                                         "unit": "GB/s", "bytes": byts}}
     return out
+
+
+# head-shaped GEMM on the unrotated group-128 grid: the pages give no vocabulary
+# size, so a round 131072 rows over the MoE layer's hidden size
+HEAD = dict(N=131072, K=2048)
 
 
 # --------------------------------------------------------------------------- profiling cases
 CASES = ("gemv_gateup_m8", "gemv_down_m8", "prefill_gateup_m512", "prefill_down_m512", "prefill_gateup_m4096",
          "prefill_down_m4096", "quant_m4096_k17408", "quant_m4096_k5120", "moe_t1", "moe_t8", "moe_t512",
-         "moe_t4096", "moe_g128_t1", "moe_g128_t8", "moe_g128_t512", "moe_g128_t4096", "hadamard_m1",
+         "moe_t4096", "moe_g128_t1", "moe_g128_t8", "moe_g128_t512", "moe_g128_t4096", "head_m1", "head_m8", "hadamard_m1",
          "hadamard_m200", "hadamard_m2048")
 
 
@@ -618,6 +644,15 @@ def run_case(name, torch, dev, reps=4):
         torch.cuda.empty_cache()
         for _ in range(reps):
             w8a8.moe_g128_forward(x, lg, q13, s13, q2, s2, k, y=y, ws=ws)
+    elif kind == "head":
+        M = int(rest[1:])
+        qw, sw = w8a8.group128_quant(randn(HEAD["N"], HEAD["K"], std=0.02).to(torch.bfloat16))
+        x = randn(M, HEAD["K"]).to(torch.bfloat16)
+        y = torch.empty((M, HEAD["N"]), dtype=torch.bfloat16, device=dev)
+        torch.cuda.empty_cache()
+        for _ in range(reps):
+            q, s = w8a8.group128_quant(x)
+            w8a8.linear_group128(q, s, qw, sw, y=y)
     elif kind == "hadamard":
         M = int(rest[1:])
         d = inputs.HADAMARD

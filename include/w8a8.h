@@ -200,9 +200,26 @@ W8A8_API int fwht128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, u
  *   y[m,n] = bf16_rne( (1/128) * sum_g float(p_g) * (sx[m,g] * sw[n,g]) ),
  *   p_g = sum over the 128 k of group g of qx[m,k] qw[n,k] (int32, exact).
  * qx int8 [M, K], sx bf16 [M, K/128], qw int8 [N, K], sw bf16 [N, K/128],
- * y bf16 [M, N].  The fp32 group sum order is unspecified. */
+ * y bf16 [M, N].  The groups are summed in ascending order, one fp32 fma
+ * each: acc = fma(float(p_g), sx * sw, acc); y = bf16_rne(acc * (1/128)).
+ * M <= 8 needs N % 16 == 0 and K <= 8192. */
 W8A8_API int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
                      int64_t M, int64_t N, int64_t K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The group-128 grid without the rotation -- [IQ8R] file table (Head: "the
+ * lm_head int8 with a bf16 scale per row and 128") and recipe row
+ * output.weight (codes=i8 group=128 scale=bf16 clamp=sym, no transform).
+ * group128_quant: fwht128_quant without the butterflies: for each 128-wide
+ * block of each row of x bf16 [M, K] (K % 128 == 0): s = bf16_rne(max|x| /
+ * 127), q = clamp(rne(x / s), -127, 127); q int8 [M, K], s bf16 [M, K/128].
+ * w8a8_linear_group128: y[m,n] = bf16_rne( sum_g float(p_g) * (sx[m,g] *
+ * sw[n,g]) ) with one fp32 fma per group in ascending g -- the group-128
+ * GEMM without the 1/128 (there is no rotation to undo).  Shapes, layouts
+ * and the M <= 8 / M > 8 split as w8a8_linear_g128. */
+W8A8_API int group128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, void* stream);
+W8A8_API int w8a8_linear_group128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw,
+                                  uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Routed experts on the FWHT128 grid -- [IQ8R] file table (Experts: int8 on

@@ -15,7 +15,8 @@
 // gemv_g128_kernel: decode-sized M (<= 8) group-scaled GEMV.  Warps split the
 // K groups, keep each group's exact int32 partial p_g in shared memory, and
 // one warp applies acc = fma(float(p_g), sx*sw, acc) in ascending g -- the
-// same fp32 steps as the serial definition.
+// same fp32 steps as the serial definition -- and y = acc * post (1/128 in the
+// rotated domain, 1 on the unrotated grid).
 #pragma once
 
 #include "common.cuh"
@@ -88,10 +89,12 @@ __device__ __forceinline__ void fwht128_load4(const float* src, float (&v)[4]) {
 }
 
 // One warp per 128-wide block of a row; bf16 rows (activations, weights) or
-// fp32 rows (the routed experts' gated intermediate).  On a chain with
-// programmatic dependent launch it waits for the kernel before it (a no-op
-// otherwise) and reads its rows with coherent loads.
-template <typename Tin>
+// fp32 rows (the routed experts' gated intermediate).  ROTATE = false is the
+// same group quantizer on the unrotated grid (the head's format: a bf16 scale
+// per row and 128 of K, no transform).  On a chain with programmatic
+// dependent launch it waits for the kernel before it (a no-op otherwise) and
+// reads its rows with coherent loads.
+template <typename Tin, bool ROTATE = true>
 __global__ void __launch_bounds__(256) fwht128_quant_kernel(const Tin* __restrict__ x, int64_t M, int64_t K,
                                                             int8_t* __restrict__ q, uint16_t* __restrict__ s) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(256) fwht128_quant_kernel(const Tin* __restric
     const int64_t m = blk / G, g = blk % G;
     float v[4];
     fwht128_load4(x + m * K + g * 128 + 4 * lane, v);
-    fwht128_warp(v, lane);
+    if constexpr (ROTATE) fwht128_warp(v, lane);
     uint16_t sb;
     const uint32_t pk = fwht128_codes(v, sb);
     *reinterpret_cast<uint32_t*>(q + m * K + g * 128 + 4 * lane) = pk;
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
                                                         const uint16_t* __restrict__ sx,
                                                         const int8_t* __restrict__ qw,
                                                         const uint16_t* __restrict__ sw, uint16_t* __restrict__ y,
-                                                        int M, int N, int K) {
+                                                        int M, int N, int K, float post) {
     __shared__ int4 pg[kG128MaxGroups][32];
     __shared__ float s_sw[16][kG128MaxGroups];   // [row in CTA][group]
     __shared__ float s_sx[8][kG128MaxGroups];    // [token][group]
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
     for (int j = 0; j < 4; ++j) {
         const int m = 2 * t + (j & 1);
         const int n = block * 16 + g8 + 8 * (j >> 1);
-        if (m < M && n < N) y[(int64_t)m * N + n] = float_to_bf16_bits(__fmul_rn(yv[j], 0.0078125f));
+        if (m < M && n < N) y[(int64_t)m * N + n] = float_to_bf16_bits(__fmul_rn(yv[j], post));
     }
 }
 

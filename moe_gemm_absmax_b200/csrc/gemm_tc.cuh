@@ -51,6 +51,7 @@ struct TcParams {
     const float* sw;        // [N]        (kEpiBf16; grouped: [E, N] per-expert channel scales)
     const uint16_t* gsx;    // [M, G] bf16 (kEpiG128)
     const uint16_t* gsw;    // [N, G] bf16 (kEpiG128)
+    float gpost;            // kEpiG128: final factor (1/128 in the rotated domain, 1 unrotated)
     void* out;              // bf16 or int32 [M, N], row stride N
     // ---- grouped (MoE) mode: A = expert-sorted rows, B = per-expert weights [E * N, K]
     const int32_t* counts;  // [E] rows of each expert
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                 }
                 if (ok && row_ok) {
                     uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
-                    const uint64_t inv2 = f2_pack(0.0078125f, 0.0078125f);
+                    const uint64_t inv2 = f2_pack(p.gpost, p.gpost);
 #pragma unroll
                     for (int i = 0; i < kChunks; ++i) {
 #pragma unroll

@@ -1138,27 +1138,21 @@ int w8a8_moe_g128_forward(const uint16_t* x, const uint16_t* logits, const int8_
     return W8A8_OK;
 }
 
-// ----------------------------------------------------------------- FWHT128
-int fwht128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, void* stream) {
-    if (!x || !q || !s || M <= 0 || K <= 0 || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 2)) return W8A8_ERR_INVALID_ARG;
-    const int64_t blocks = M * (K / 128);
-    const int64_t ctas = (blocks + 7) / 8;
-    if (ctas > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
-    fwht128_quant_kernel<<<(unsigned)ctas, 256, 0, (cudaStream_t)stream>>>(x, M, K, q, s);
-    return last_launch_status();
-}
+}  // extern "C"
 
-int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
-                     int64_t M, int64_t N, int64_t K, void* stream) {
+// ----------------------------------------------------------------- FWHT128 and the unrotated group-128 grid
+namespace {
+// The group-128 GEMM of the rotated domain (post = 1/128) and of the
+// unrotated grid (post = 1).
+int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
+                        int64_t M, int64_t N, int64_t K, float post, cudaStream_t st) {
     if (!qx || !sx || !qw || !sw || !y) return W8A8_ERR_INVALID_ARG;
     if (!gemm_shape_ok(M, N, K) || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
     if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sx, 2) || !aligned(sw, 2))
         return W8A8_ERR_INVALID_ARG;
-    cudaStream_t st = (cudaStream_t)stream;
     if (M <= 8) {
         if (K / 128 > kG128MaxGroups || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
-        gemv_g128_kernel<<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K);
+        gemv_g128_kernel<<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post);
         return last_launch_status();
     }
     TcParams p = {};
@@ -1167,8 +1161,43 @@ int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, con
     p.K = (int)K;
     p.gsx = sx;
     p.gsw = sw;
+    p.gpost = post;
     p.out = y;
     return launch_tc<128, 6, kEpiG128, 4, 8>(qx, qw, p, st);
+}
+
+int group_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, bool rotate, cudaStream_t st) {
+    if (!x || !q || !s || M <= 0 || K <= 0 || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 2)) return W8A8_ERR_INVALID_ARG;
+    const int64_t blocks = M * (K / 128);
+    const int64_t ctas = (blocks + 7) / 8;
+    if (ctas > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
+    if (rotate)
+        fwht128_quant_kernel<uint16_t, true><<<(unsigned)ctas, 256, 0, st>>>(x, M, K, q, s);
+    else
+        fwht128_quant_kernel<uint16_t, false><<<(unsigned)ctas, 256, 0, st>>>(x, M, K, q, s);
+    return last_launch_status();
+}
+}  // namespace
+
+extern "C" {
+
+int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
+                     int64_t M, int64_t N, int64_t K, void* stream) {
+    return linear_group_scaled(qx, sx, qw, sw, y, M, N, K, 0.0078125f, (cudaStream_t)stream);
+}
+
+int fwht128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, void* stream) {
+    return group_quant(x, M, K, q, s, true, (cudaStream_t)stream);
+}
+
+int group128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, void* stream) {
+    return group_quant(x, M, K, q, s, false, (cudaStream_t)stream);
+}
+
+int w8a8_linear_group128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
+                         int64_t M, int64_t N, int64_t K, void* stream) {
+    return linear_group_scaled(qx, sx, qw, sw, y, M, N, K, 1.0f, (cudaStream_t)stream);
 }
 
 // ----------------------------------------------------------------- diagnostics

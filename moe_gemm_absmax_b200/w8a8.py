@@ -25,6 +25,7 @@ EXPORTS = (
     "w8a8_linear_noalloc_scratch_size", "w8a8_linear_noalloc",
     "w8a8_gemm_workspace_size", "w8a8_gemm_q", "w8a8_gemm_s32", "w8a8_moe_workspace_size",
     "w8a8_moe_forward", "w8a8_moe_g128_workspace_size", "w8a8_moe_g128_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
+    "group128_quant", "w8a8_linear_group128",
     "w8a8_exp_proj",
     "w8a8_get_device_error", "w8a8_debug_wait_timeout", "w8a8_status_str", "w8a8_version",
 )
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         "w8a8_mlp_forward": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, ctypes.POINTER(MlpDebug), vp], i32),
         "fwht128_quant": ([vp, i64, i64, vp, vp, vp], i32),
         "w8a8_linear_g128": ([vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
+        "group128_quant": ([vp, i64, i64, vp, vp, vp], i32),
+        "w8a8_linear_group128": ([vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "w8a8_exp_proj": ([vp, vp, i64, vp], i32),
         "w8a8_get_device_error": ([vp, ctypes.POINTER(ctypes.c_int)], i32),
         "w8a8_debug_wait_timeout": ([i64, vp], i32),
@@ -385,6 +388,32 @@ def linear_g128(qx, sx, qw, sw, y=None, stream=None) -> torch.Tensor:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
     _check(lib().w8a8_linear_g128(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(y), M, N, K, _stream(stream)),
            "w8a8_linear_g128")
+    return y
+
+
+def group128_quant(x: torch.Tensor, stream=None):
+    """Group-128 quant without the rotation (the head's grid): bf16 x [M,K] ->
+    (int8 [M,K], bf16 scales [M,K/128])."""
+    _need(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s = torch.empty((M, K // 128), dtype=torch.bfloat16, device=x.device)
+    _check(lib().group128_quant(_ptr(x), M, K, _ptr(q), _ptr(s), _stream(stream)), "group128_quant")
+    return q, s
+
+
+def linear_group128(qx, sx, qw, sw, y=None, stream=None) -> torch.Tensor:
+    """Group-128 GEMM on the unrotated grid (no 1/128): -> bf16 y [M,N]."""
+    _need(qx, torch.int8, "qx", 2)
+    _need(qw, torch.int8, "qw", 2)
+    _need(sx, torch.bfloat16, "sx", 2)
+    _need(sw, torch.bfloat16, "sw", 2)
+    M, K = qx.shape
+    N = qw.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+    _check(lib().w8a8_linear_group128(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(y), M, N, K, _stream(stream)),
+           "w8a8_linear_group128")
     return y
 
 

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _declared():
     src = open(os.path.join(ROOT, "include", "w8a8.h")).read()
-    return sorted(set(re.findall(r"^W8A8_API\s+[\w\s\*]+?\b((?:w8a8|fwht128)_\w+)\s*\(", src, re.M)))
+    return sorted(set(re.findall(r"^W8A8_API\s+[\w\s\*]+?\b((?:w8a8|fwht128|group128)_\w+)\s*\(", src, re.M)))
 
 
 @pytest.fixture(scope="module")

@@ -48,3 +48,43 @@ def test_linear_g128(orc, M):
     yo, y32 = orc.gemm_g128(qxo[rows], sxo[rows], qwo, swo)
     exact = assert_bf16_close(y[rows], y32, what=f"g128 M={M}")
     assert exact == 1.0
+
+
+# ---- the unrotated group-128 grid (the head's format: a bf16 scale per row and 128, no transform)
+
+@pytest.mark.parametrize("M", [1, 3, 2048])
+def test_group128_quant_bit_exact(orc, M):
+    xb, wb = inputs.hadamard_linear(M + 3, M)
+    xb = xb.copy()
+    xb[0, 256:384] = 0   # a zero block
+    q, s = w8a8.group128_quant(to_dev_bf16(xb))
+    qo, so = orc.group128_quant(xb)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(from_dev_bf16(s), so)
+
+
+@pytest.mark.parametrize("M,N", [(1, 4096), (4, 4096), (8, 1040), (9, 4096), (200, 1040), (2048, 4096)])
+def test_linear_group128(orc, M, N):
+    xb, wb = inputs.hadamard_linear(M + 29, M, N=N)
+    qx, sx = w8a8.group128_quant(to_dev_bf16(xb))
+    qw, sw = w8a8.group128_quant(to_dev_bf16(wb))
+    y = from_dev_bf16(w8a8.linear_group128(qx, sx, qw, sw))
+    qxo, sxo = orc.group128_quant(xb)
+    qwo, swo = orc.group128_quant(wb)
+    assert np.array_equal(qw.cpu().numpy(), qwo) and np.array_equal(from_dev_bf16(sw), swo)
+    rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 48),
+                                                                  [0, 127, 128, M - 1]]))
+    yo, y32 = orc.gemm_group128(qxo[rows], sxo[rows], qwo, swo)
+    assert assert_bf16_close(y[rows], y32, what=f"group128 M={M}") == 1.0
+    assert np.array_equal(y[rows], yo)
+
+
+def test_linear_group128_is_128x_the_rotated_form():
+    """Same codes and scales through both entry points: the unrotated GEMM is
+    the rotated one without its 1/128 (bit for bit in fp32, so after bf16 too)."""
+    xb, wb = inputs.hadamard_linear(3, 16, N=512)
+    qx, sx = w8a8.group128_quant(to_dev_bf16(xb))
+    qw, sw = w8a8.group128_quant(to_dev_bf16(wb))
+    a = w8a8.linear_group128(qx, sx, qw, sw).float()
+    b = w8a8.linear_g128(qx, sx, qw, sw).float()
+    assert torch.equal(a, b * 128)
