@@ -82,6 +82,10 @@ def lib():
             L.oracle_gemm_g128.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             L.oracle_fwht128_quant_f32.argtypes = [vp, i64, i64, vp, vp]
             L.oracle_group128_quant.argtypes = [vp, i64, i64, vp, vp]
+            L.oracle_trunk_weight_quant.argtypes = [vp, i64, i64, vp, vp, vp]
+            L.oracle_gemm_trunk.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
+            L.oracle_shared_expert_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32,
+                                                       vp, vp, vp, vp, vp, vp]
             L.oracle_gemm_group128.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             L.oracle_moe_g128_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32,
                                                   vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -365,6 +369,54 @@ def gemm_group128(qx, sx_bits, qw, sw_bits):
     y32 = np.empty((M, N), np.float32)
     lib().oracle_gemm_group128(_p(qx), _p(sx), _p(qw), _p(sw), M, N, K, _p(y), _p(y32))
     return y, y32
+
+
+def trunk_weight_quant(w_bits):
+    """Two-level trunk format of bf16 rows [N,K] (K % 256 == 0): returns
+    (codes int8 [N,K], u8 group scales [N,K/256], bf16 row scales [N])."""
+    w = _c(w_bits, np.uint16)
+    N, K = w.shape
+    assert K % 256 == 0
+    q = np.empty((N, K), np.int8)
+    su8 = np.empty((N, K // 256), np.uint8)
+    s2 = np.empty(N, np.uint16)
+    lib().oracle_trunk_weight_quant(_p(w), N, K, _p(q), _p(su8), _p(s2))
+    return q, su8, s2
+
+
+def gemm_trunk(qx, sx_bits, qw, su8, s2_bits):
+    """Trunk GEMM (x rotated with bf16 group-128 scales, W two-level): returns
+    (y bf16 bits [M,N], y fp32)."""
+    qx, qw = _c(qx, np.int8), _c(qw, np.int8)
+    sx, su8, s2 = _c(sx_bits, np.uint16), _c(su8, np.uint8), _c(s2_bits, np.uint16)
+    M, K = qx.shape
+    N = qw.shape[0]
+    y = np.empty((M, N), np.uint16)
+    y32 = np.empty((M, N), np.float32)
+    lib().oracle_gemm_trunk(_p(qx), _p(sx), _p(qw), _p(su8), _p(s2), M, N, K, _p(y), _p(y32))
+    return y, y32
+
+
+def shared_expert_forward(x_bits, w13, u13, r13_bits, w2, s2_bits):
+    """The shared expert on the rotated grid: x bf16 bits [M,H]; gate_up in the
+    trunk format (w13 int8 [2I,H], u8 [2I,H/256], bf16 row scales [2I]); down
+    on the group-128 grid (w2 int8 [H,I], bf16 [H,I/128]).  Returns a dict
+    with y (bf16 bits), y32, qx, sx, qa, sa (scales as bf16 bits)."""
+    x = _c(x_bits, np.uint16)
+    w13, w2 = _c(w13, np.int8), _c(w2, np.int8)
+    u13, r13, s2 = _c(u13, np.uint8), _c(r13_bits, np.uint16), _c(s2_bits, np.uint16)
+    M, H = x.shape
+    I2 = w13.shape[0]
+    I = I2 // 2
+    assert w13.shape == (I2, H) and u13.shape == (I2, H // 256) and r13.shape == (I2,)
+    assert w2.shape == (H, I) and s2.shape == (H, I // 128)
+    out = dict(y=np.empty((M, H), np.uint16), y32=np.empty((M, H), np.float32),
+               qx=np.empty((M, H), np.int8), sx=np.empty((M, H // 128), np.uint16),
+               qa=np.empty((M, I), np.int8), sa=np.empty((M, I // 128), np.uint16))
+    lib().oracle_shared_expert_forward(_p(x), _p(w13), _p(u13), _p(r13), _p(w2), _p(s2), M, H, I,
+                                       _p(out["y"]), _p(out["y32"]), _p(out["qx"]), _p(out["sx"]),
+                                       _p(out["qa"]), _p(out["sa"]))
+    return out
 
 
 def set_threads(n: int) -> None:

@@ -604,6 +604,92 @@ void oracle_gemm_group128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, 
 }
 
 /* ------------------------------------------------------------------ */
+/* f4: the trunk linears' two-level scales ([IQ8R] file table, Trunk:    */
+/* int8 codes -127..127 "with a u8 scale per row and 256 of K under a    */
+/* bf16 scale a row, each 128 of K rotated by the unnormalised          */
+/* Hadamard, round to nearest"; recipe: codes=i8 group=256 scale=u8      */
+/* scale2=bf16 block2=1x* transform=fwht128 clamp=sym rule=search).      */
+/* Per row n of W (bf16 [N, K], K % 256 == 0), after the rotation of     */
+/* each 128 of K:                                                         */
+/*   scale2 = bf16_rne(max |w'| / (127 * 255))                            */
+/*   for each 256-wide group j, u8[j] = the u in 1..255 whose scale      */
+/*   s = float(u) * float(scale2) gives the smallest largest error        */
+/*   max_k |w'_k - q_k * s|, q_k = clamp(rne(w'_k / s), +-127) (fp32,     */
+/*   one rounding per operation; ties to the smaller u)                   */
+/*   codes from the chosen s.  A zero row: scale2 = 0, u8 = 0, codes 0.   */
+/* ------------------------------------------------------------------ */
+static float trunk_group_error(const float* v, float s)
+{
+    float worst = 0.0f;
+    for (int k = 0; k < 256; ++k) {
+        int8_t c = clamp_sym127(rne_to_int(v[k] / s));
+        float e = fabsf(v[k] - (float)c * s);
+        if (e > worst) worst = e;
+    }
+    return worst;
+}
+
+void oracle_trunk_weight_quant(const bf16_t* w, int64_t N, int64_t K, int8_t* q, uint8_t* su8, bf16_t* s2)
+{
+    const int64_t G2 = K / 256;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; ++n) {
+        float* v = (float*)malloc(sizeof(float) * (size_t)K);
+        for (int64_t k = 0; k < K; ++k) v[k] = oracle_bf16_to_f32(w[n * K + k]);
+        for (int64_t g = 0; g < K / 128; ++g) oracle_fwht128(v + g * 128);
+        float rmax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) { float a = fabsf(v[k]); if (a > rmax) rmax = a; }
+        bf16_t sb = oracle_f32_to_bf16(rmax / 32385.0f);
+        float s2f = oracle_bf16_to_f32(sb);
+        s2[n] = sb;
+        for (int64_t j = 0; j < G2; ++j) {
+            const float* vg = v + j * 256;
+            int best = 0;
+            if (s2f != 0.0f) {
+                float best_err = INFINITY;
+                for (int u = 1; u <= 255; ++u) {
+                    float e = trunk_group_error(vg, (float)u * s2f);
+                    if (e < best_err) { best_err = e; best = u; }
+                }
+            }
+            su8[n * G2 + j] = (uint8_t)best;
+            float s = (float)best * s2f;
+            for (int k = 0; k < 256; ++k)
+                q[n * K + j * 256 + k] = best ? clamp_sym127(rne_to_int(vg[k] / s)) : 0;
+        }
+        free(v);
+    }
+}
+
+/* The trunk GEMM: x on the rotated grid of a12 (bf16 scale per token and  */
+/* 128 of K), W in the two-level format above:                             */
+/*   sw_g = float(u8[n, g / 2]) * float(scale2[n])      (exact in fp32)      */
+/*   acc  = fma(float(p_g), float(sx[m, g]) * sw_g, acc), g ascending        */
+/*   y    = bf16_rne(acc * (1/128))                                          */
+void oracle_gemm_trunk(const int8_t* qx, const bf16_t* sx, const int8_t* qw, const uint8_t* su8,
+                       const bf16_t* s2, int64_t M, int64_t N, int64_t K, bf16_t* y, float* y32)
+{
+    int64_t G = K / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int64_t g = 0; g < G; ++g) {
+                int32_t p = 0;
+                for (int k = 0; k < 128; ++k)
+                    p += (int32_t)qx[m * K + g * 128 + k] * (int32_t)qw[n * K + g * 128 + k];
+                float swg = (float)su8[n * (K / 256) + g / 2] * oracle_bf16_to_f32(s2[n]);
+                float sc = oracle_bf16_to_f32(sx[m * G + g]) * swg;
+                acc = fmaf((float)p, sc, acc);
+            }
+            float r = acc * 0.0078125f;
+            if (y) y[m * N + n] = oracle_f32_to_bf16(r);
+            if (y32) y32[m * N + n] = r;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* f1: routed experts on the rotated grid ([IQ8R] file table: "Experts   */
 /* ... int8 on the same rotated grid with a bf16 scale per row and 128  */
 /* of K"; "Activations int8 under the same rotation, the routed experts  */
@@ -695,6 +781,53 @@ void oracle_moe_g128_forward(const bf16_t* x, const bf16_t* logits,
         if (qx_out) memcpy(qx_out + i * H, qx, (size_t)H);
         if (sx_out) memcpy(sx_out + i * GH, sx, sizeof(bf16_t) * (size_t)GH);
         free(ids); free(wts); free(qx); free(sx); free(v); free(a); free(qa); free(sa); free(out); free(oabs);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* f3: the shared expert ([IQ8R] file table, Experts: "the shared expert  */
+/* likewise (its gate/up projection as the trunk's linears)"; recipe rows */
+/* ffn_gate_up_shexp: the trunk's two-level format, ffn_down_shexp:       */
+/* group=128 scale=bf16 transform=fwht128).  A dense gated MLP on the     */
+/* rotated grid, for each token m:                                         */
+/*   (qx, sx[g]) = fwht128_quant(x[m])                                     */
+/*   v_r = the trunk product of (qx, sx) with (w13[r], u8[r], scale2[r])   */
+/*   a_i = SiLU(v_2i) * v_2i+1                                             */
+/*   (qa, sa[g]) = fwht128_quant(a)               (rotation along I, fp32) */
+/*   y_n = bf16( g128(qa, sa; w2[n], s2[n]) )                              */
+/* w13 int8 [2I, H] + u8 [2I, H/256] + bf16 [2I]; w2 int8 [H, I] + bf16   */
+/* [H, I/128].                                                             */
+/* ------------------------------------------------------------------ */
+void oracle_shared_expert_forward(const bf16_t* x, const int8_t* w13, const uint8_t* u13, const bf16_t* r13,
+                                  const int8_t* w2, const bf16_t* s2, int64_t M, int H, int I,
+                                  bf16_t* y, float* y32, int8_t* qx_out, bf16_t* sx_out,
+                                  int8_t* qa_out, bf16_t* sa_out)
+{
+    const int GH = H / 128, GI = I / 128;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        int8_t* qx = (int8_t*)malloc((size_t)H);
+        bf16_t* sx = (bf16_t*)malloc(sizeof(bf16_t) * (size_t)GH);
+        float* v = (float*)malloc(sizeof(float) * (size_t)(2 * I));
+        float* a = (float*)malloc(sizeof(float) * (size_t)I);
+        int8_t* qa = (int8_t*)malloc((size_t)I);
+        bf16_t* sa = (bf16_t*)malloc(sizeof(bf16_t) * (size_t)GI);
+        oracle_fwht128_quant(x + m * H, 1, H, qx, sx, NULL);
+        for (int r = 0; r < 2 * I; ++r)
+            oracle_gemm_trunk(qx, sx, w13 + (int64_t)r * H, u13 + (int64_t)r * (H / 256), r13 + r, 1, 1, H,
+                              NULL, v + r);
+        for (int i = 0; i < I; ++i) a[i] = oracle_silu(v[2 * i]) * v[2 * i + 1];
+        oracle_fwht128_quant_f32(a, 1, I, qa, sa);
+        for (int n = 0; n < H; ++n) {
+            float yn = g128_dot(qa, sa, w2 + (int64_t)n * I, s2 + (int64_t)n * GI, I);
+            if (y) y[m * H + n] = oracle_f32_to_bf16(yn);
+            if (y32) y32[m * H + n] = yn;
+        }
+        if (qx_out) memcpy(qx_out + m * H, qx, (size_t)H);
+        if (sx_out) memcpy(sx_out + m * GH, sx, sizeof(bf16_t) * (size_t)GH);
+        if (qa_out) memcpy(qa_out + m * I, qa, (size_t)I);
+        if (sa_out) memcpy(sa_out + m * GI, sa, sizeof(bf16_t) * (size_t)GI);
+        free(qx); free(sx); free(v); free(a); free(qa); free(sa);
     }
 }
 
