@@ -222,6 +222,57 @@ W8A8_API int w8a8_linear_group128(const int8_t* qx, const uint16_t* sx, const in
                                   uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The trunk linears' two-level format -- [IQ8R] file table (Trunk: int8
+ * codes -127..127 "with a u8 scale per row and 256 of K under a bf16 scale a
+ * row, each 128 of K rotated by the unnormalised Hadamard, round to nearest")
+ * and recipe (codes=i8 group=256 scale=u8 scale2=bf16 block2=1x*
+ * transform=fwht128 clamp=sym rule=search).
+ * w8a8_trunk_weight_quant (set-up): each row of w bf16 [N, K] (K % 256 == 0,
+ * K <= 8192) rotated 128 at a time; scale2[n] = bf16_rne(max|w'| / (127*255));
+ * for each 256-wide group j, su8[n, j] = the u in 1..255 whose scale
+ * s = u * scale2 gives the smallest largest error max_k |w'_k - q_k s| with
+ * q_k = clamp(rne(w'_k / s), +-127) (ties to the smaller u); codes under the
+ * chosen s.  A zero row: scale2 = 0, su8 = 0, codes 0.
+ *   q int8 [N, K];  su8 uint8 [N, K/256];  s2 bf16 [N].
+ * w8a8_linear_trunk: x codes and bf16 group scales from fwht128_quant
+ * (qx int8 [M, K], sx bf16 [M, K/128]) times W in that format:
+ *   y[m,n] = bf16_rne( (1/128) * sum_g fma(float(p_g), sx[m,g] * sw_g, .) ),
+ *   sw_g = float(su8[n, g/2]) * float(s2[n]) (exact), groups ascending.
+ * M <= 8 runs the GEMV (N % 16 == 0), larger M the tcgen05 GEMM. */
+W8A8_API int w8a8_trunk_weight_quant(const uint16_t* w, int64_t N, int64_t K, int8_t* q, uint8_t* su8, uint16_t* s2,
+                                     void* stream);
+W8A8_API int w8a8_linear_trunk(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint8_t* su8,
+                               const uint16_t* s2, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The shared expert -- [IQ8R] file table (Experts: "the shared expert
+ * likewise (its gate/up projection as the trunk's linears)") and recipe rows
+ * ffn_gate_up_shexp (the trunk format above) and ffn_down_shexp (group=128
+ * scale=bf16 transform=fwht128).  A dense gated MLP on the rotated grid:
+ *   x    bf16 [M, H]
+ *   w13  int8 [2I, H] + su8 [2I, H/256] + bf16 row scales [2I] (trunk format;
+ *        row 2i = gate_i, 2i+1 = up_i)
+ *   w2   int8 [H, I] + bf16 [H, I/128] (fwht128_quant of the bf16 rows)
+ *   y    bf16 [M, H]
+ * Steps: (qx, sx) = fwht128_quant(x); v = the trunk product of (qx, sx) with
+ * w13 (fp32); a_i = SiLU(v_2i) * v_2i+1; (qa, sa) = FWHT128 group quant of the
+ * fp32 row a (along I); y = bf16( the group-128 product of (qa, sa) with w2 ).
+ * Requires H % 256 == 0, H <= 4096, I % 128 == 0, I <= 2048; 16-byte aligned
+ * x, w13, w2, y; 256-byte aligned ws; ws_bytes >=
+ * w8a8_shared_expert_workspace_size(M, H, I).  `dbg` may be NULL. */
+typedef struct w8a8_shared_expert_debug {
+    int8_t* qx;          /* [M, H] rotated codes of x */
+    uint16_t* sx;        /* [M, H/128] bf16 */
+    int8_t* qa;          /* [M, I] rotated codes of the gated intermediate */
+    uint16_t* sa;        /* [M, I/128] bf16 */
+} w8a8_shared_expert_debug;
+
+W8A8_API size_t w8a8_shared_expert_workspace_size(int64_t M, int H, int I);
+W8A8_API int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8_t* u13, const uint16_t* r13,
+                                        const int8_t* w2, const uint16_t* s2, uint16_t* y, int64_t M, int H, int I,
+                                        void* ws, size_t ws_bytes, const w8a8_shared_expert_debug* dbg, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Routed experts on the FWHT128 grid -- [IQ8R] file table (Experts: int8 on
  * the same rotated grid with a bf16 scale per row and 128 of K; Activations:
  * int8 under the same rotation, the routed experts reading the codes the

@@ -122,7 +122,9 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
                                                         const uint16_t* __restrict__ sx,
                                                         const int8_t* __restrict__ qw,
                                                         const uint16_t* __restrict__ sw, uint16_t* __restrict__ y,
-                                                        int M, int N, int K, float post) {
+                                                        int M, int N, int K, float post,
+                                                        const uint8_t* __restrict__ sw_u8,
+                                                        const uint16_t* __restrict__ sw_row) {
     __shared__ int4 pg[kG128MaxGroups][32];
     __shared__ float s_sw[16][kG128MaxGroups];   // [row in CTA][group]
     __shared__ float s_sx[8][kG128MaxGroups];    // [token][group]
@@ -132,7 +134,11 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
     const int block = blockIdx.x;
     for (int i = threadIdx.x; i < 16 * G; i += blockDim.x) {
         const int r = i / G, grp = i - r * G, n = block * 16 + r;
-        s_sw[r][grp] = n < N ? bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp)) : 0.0f;
+        float v = 0.0f;
+        if (n < N)   // the two-level trunk format: u8 per 256 of K times a bf16 row scale (exact)
+            v = sw_u8 ? __fmul_rn((float)__ldg(sw_u8 + (int64_t)n * (G / 2) + grp / 2), bf16_bits_to_float(__ldg(sw_row + n)))
+                      : bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp));
+        s_sw[r][grp] = v;
     }
     for (int i = threadIdx.x; i < 8 * G; i += blockDim.x) {
         const int m = i / G, grp = i - m * G;

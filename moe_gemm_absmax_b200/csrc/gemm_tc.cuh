@@ -52,6 +52,8 @@ struct TcParams {
     const uint16_t* gsx;    // [M, G] bf16 (kEpiG128)
     const uint16_t* gsw;    // [N, G] bf16 (kEpiG128)
     float gpost;            // kEpiG128: final factor (1/128 in the rotated domain, 1 unrotated)
+    const uint8_t* gsw_u8;  // kEpiG128, two-level trunk format: [N, G / 2] u8 ...
+    const uint16_t* gsw_row;// ... times a bf16 row scale [N] (gsw unused)
     void* out;              // bf16 or int32 [M, N], row stride N
     // ---- grouped (MoE) mode: A = expert-sorted rows, B = per-expert weights [E * N, K]
     const int32_t* counts;  // [E] rows of each expert
@@ -308,6 +310,14 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                 const int G = p.num_k_blocks;
                 const uint64_t magic2 = 0x4B4000004B400000ull;
                 float* wsc = epi_scratch + (warp - 2) * 64;
+                // column scale of group g: bf16, or (trunk format) u8 per 256 of K times a bf16 row scale
+                auto col_scale = [&](int col, int g) -> float {
+                    if (col >= p.N) return 0.0f;
+                    if (p.gsw_u8)
+                        return __fmul_rn((float)__ldg(p.gsw_u8 + (int64_t)col * (G / 2) + g / 2),
+                                         bf16_bits_to_float(__ldg(p.gsw_row + col)));
+                    return bf16_bits_to_float(__ldg(p.gsw + (int64_t)col * G + g));
+                };
                 uint64_t y2[kChunks * 16];
 #pragma unroll
                 for (int j = 0; j < kChunks * 16; ++j) y2[j] = 0ull;
@@ -316,7 +326,7 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
 #pragma unroll
                 for (int i = 0; i < kChunks; ++i) {
                     const int col = nt * BN + c0 + i * kStep + lane;
-                    sw_next[i] = col < p.N ? bf16_bits_to_float(__ldg(p.gsw + (int64_t)col * G)) : 0.0f;
+                    sw_next[i] = col_scale(col, 0);
                 }
                 for (int kb = 0; kb < G; ++kb) {
                     const float sxg = sx_next;
@@ -329,7 +339,7 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
 #pragma unroll
                         for (int i = 0; i < kChunks; ++i) {
                             const int col = nt * BN + c0 + i * kStep + lane;
-                            sw_next[i] = col < p.N ? bf16_bits_to_float(__ldg(p.gsw + (int64_t)col * G + kb + 1)) : 0.0f;
+                            sw_next[i] = col_scale(col, kb + 1);
                         }
                     }
                     if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) {

@@ -87,6 +87,8 @@ struct MoeSwapArgs {
     // group-128 form (K / 128 groups, bf16 scales)
     const uint16_t* gsw;      // [E * rows, K / 128]
     const uint16_t* gsx;      // [R, K / 128] of the sorted rows
+    const uint8_t* gsw_u8;    // two-level trunk format instead of gsw: [E * rows, K / 256] u8 ...
+    const uint16_t* gsw_row;  // ... times a bf16 row scale [E * rows]
 };
 
 // Token block b (in tile_off numbering) -> expert, first sorted row, rows;
@@ -382,15 +384,22 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             ms_epi_sync<256>();   // also: every warp is done with this buffer's use two units ago
             buf ^= 1;
             const int n = g * kMsBM + quarter * 32 + lane;   // weight row of expert e
-            const uint16_t* swrow = a.gsw + ((int64_t)k.e * a.rows + n) * G;
-            float sw_next = bf16_bits_to_float(__ldg(swrow));
+            const int64_t wr = (int64_t)k.e * a.rows + n;
+            const uint16_t* swrow = a.gsw + wr * G;
+            // weight scale of group kb: bf16, or (trunk format) u8 per 256 of K times a bf16 row scale
+            const uint8_t* swu8 = a.gsw_u8 ? a.gsw_u8 + wr * (G / 2) : nullptr;
+            const float swr = a.gsw_u8 ? bf16_bits_to_float(__ldg(a.gsw_row + wr)) : 0.0f;
+            auto wscale = [&](int kb) -> float {
+                return swu8 ? __fmul_rn((float)__ldg(swu8 + kb / 2), swr) : bf16_bits_to_float(__ldg(swrow + kb));
+            };
+            float sw_next = wscale(0);
             uint64_t y2[HC / 2];
 #pragma unroll
             for (int i = 0; i < HC / 2; ++i) y2[i] = 0ull;
             bool ok = true;
             for (int kb = 0; kb < G; ++kb) {
                 const float swg = sw_next;
-                if (kb + 1 < G) sw_next = bf16_bits_to_float(__ldg(swrow + kb + 1));
+                if (kb + 1 < G) sw_next = wscale(kb + 1);
                 if (!mbar_wait_bounded(&tfull[slot], sphase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) {
                     ok = false;
                     break;

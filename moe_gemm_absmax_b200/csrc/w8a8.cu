@@ -19,6 +19,7 @@
 #include "moe_g128.cuh"
 #include "moe_swap.cuh"
 #include "quant.cuh"
+#include "trunk.cuh"
 #include "w8a8.h"
 
 using namespace w8a8;
@@ -1144,15 +1145,20 @@ int w8a8_moe_g128_forward(const uint16_t* x, const uint16_t* logits, const int8_
 namespace {
 // The group-128 GEMM of the rotated domain (post = 1/128) and of the
 // unrotated grid (post = 1).
+// The weight scales are bf16 per row and 128 of K (sw), or, for the trunk
+// format, u8 per row and 256 of K times a bf16 row scale (sw_u8, sw_row).
 int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
-                        int64_t M, int64_t N, int64_t K, float post, cudaStream_t st) {
-    if (!qx || !sx || !qw || !sw || !y) return W8A8_ERR_INVALID_ARG;
-    if (!gemm_shape_ok(M, N, K) || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
-    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sx, 2) || !aligned(sw, 2))
+                        int64_t M, int64_t N, int64_t K, float post, cudaStream_t st,
+                        const uint8_t* sw_u8 = nullptr, const uint16_t* sw_row = nullptr) {
+    if (!qx || !sx || !qw || !(sw || (sw_u8 && sw_row)) || !y) return W8A8_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(M, N, K) || K % (sw_u8 ? 256 : 128) != 0) return W8A8_ERR_INVALID_ARG;
+    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sx, 2) || !aligned(sw, 2) ||
+        !aligned(sw_row, 2))
         return W8A8_ERR_INVALID_ARG;
     if (M <= 8) {
         if (K / 128 > kG128MaxGroups || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
-        gemv_g128_kernel<<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post);
+        gemv_g128_kernel<<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post, sw_u8,
+                                                             sw_row);
         return last_launch_status();
     }
     TcParams p = {};
@@ -1161,6 +1167,8 @@ int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, 
     p.K = (int)K;
     p.gsx = sx;
     p.gsw = sw;
+    p.gsw_u8 = sw_u8;
+    p.gsw_row = sw_row;
     p.gpost = post;
     p.out = y;
     return launch_tc<128, 6, kEpiG128, 4, 8>(qx, qw, p, st);
@@ -1198,6 +1206,152 @@ int group128_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t*
 int w8a8_linear_group128(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint16_t* sw, uint16_t* y,
                          int64_t M, int64_t N, int64_t K, void* stream) {
     return linear_group_scaled(qx, sx, qw, sw, y, M, N, K, 1.0f, (cudaStream_t)stream);
+}
+
+// ----------------------------------------------------------------- trunk format, shared expert
+int w8a8_trunk_weight_quant(const uint16_t* w, int64_t N, int64_t K, int8_t* q, uint8_t* su8, uint16_t* s2,
+                            void* stream) {
+    if (!w || !q || !su8 || !s2 || N <= 0 || K <= 0 || K % 256 != 0) return W8A8_ERR_INVALID_ARG;
+    if (K > kTrunkMaxK || N > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
+    if (!aligned(w, 16) || !aligned(s2, 2)) return W8A8_ERR_INVALID_ARG;
+    trunk_weight_quant_kernel<<<(unsigned)N, 256, 0, (cudaStream_t)stream>>>(w, K, q, su8, s2);
+    return last_launch_status();
+}
+
+}  // extern "C"
+
+namespace {
+struct SharedWs {
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* tile_off;
+    int32_t* row_tok;
+    int32_t* row_slot;
+    float* row_w;
+    int8_t* xq;       // [M, H] rotated codes of x
+    uint16_t* sxg;    // [M, H / 128]
+    float* a;         // [M, I] fp32 gated intermediate
+    int8_t* qa;       // [M, I]
+    uint16_t* sag;    // [M, I / 128]
+    float* out;       // [M, H] fp32 before the bf16 rounding
+    size_t bytes;
+};
+
+SharedWs shared_carve(void* base, int64_t M, int H, int I) {
+    SharedWs w;
+    uint8_t* p = reinterpret_cast<uint8_t*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* r = p ? p + o : nullptr;
+        o += align_up(bytes, 256);
+        return r;
+    };
+    w.counts = reinterpret_cast<int32_t*>(take(16));
+    w.offsets = reinterpret_cast<int32_t*>(take(16));
+    w.tile_off = reinterpret_cast<int32_t*>(take(16));
+    w.row_tok = reinterpret_cast<int32_t*>(take((size_t)M * 4));
+    w.row_slot = reinterpret_cast<int32_t*>(take((size_t)M * 4));
+    w.row_w = reinterpret_cast<float*>(take((size_t)M * 4));
+    w.xq = reinterpret_cast<int8_t*>(take((size_t)M * H));
+    w.sxg = reinterpret_cast<uint16_t*>(take((size_t)M * (H / 128) * 2));
+    w.a = reinterpret_cast<float*>(take((size_t)M * I * 4));
+    w.qa = reinterpret_cast<int8_t*>(take((size_t)M * I));
+    w.sag = reinterpret_cast<uint16_t*>(take((size_t)M * (I / 128) * 2));
+    w.out = reinterpret_cast<float*>(take((size_t)M * H * 4));
+    w.bytes = o;
+    return w;
+}
+}  // namespace
+
+extern "C" {
+
+size_t w8a8_shared_expert_workspace_size(int64_t M, int H, int I) {
+    if (M <= 0 || H < 256 || I < 128) return 0;
+    return shared_carve(nullptr, M, H, I).bytes;
+}
+
+int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8_t* u13, const uint16_t* r13,
+                               const int8_t* w2, const uint16_t* s2, uint16_t* y, int64_t M, int H, int I, void* ws,
+                               size_t ws_bytes, const w8a8_shared_expert_debug* dbg, void* stream) {
+    if (!x || !w13 || !u13 || !r13 || !w2 || !s2 || !y || !ws) return W8A8_ERR_INVALID_ARG;
+    if (M <= 0 || H <= 0 || I <= 0) return W8A8_ERR_INVALID_ARG;
+    if (H % 256 != 0 || H > 128 * kMoeG128MaxGroupsH || I % 128 != 0 || I > 2048) return W8A8_ERR_UNSUPPORTED;
+    if (M > (int64_t)1 << 30) return W8A8_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(w13, 16) || !aligned(r13, 2) || !aligned(w2, 16) || !aligned(s2, 2) ||
+        !aligned(y, 16) || !aligned(ws, 256))
+        return W8A8_ERR_INVALID_ARG;
+    if (ws_bytes < w8a8_shared_expert_workspace_size(M, H, I)) return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    SharedWs w = shared_carve(ws, M, H, I);
+    int rc;
+    const int bn = M <= 12 ? 16 : (M <= 24 ? 32 : 64);
+    shared_plan_kernel<<<(unsigned)((M + 255) / 256), 256, 0, st>>>((int)M, bn, w.counts, w.offsets, w.tile_off,
+                                                                     w.row_tok, w.row_slot, w.row_w);
+    if ((rc = last_launch_status()) != W8A8_OK) return rc;
+    // x rotated along H and group-quantized: the sorted rows are the tokens
+    rc = launch_chained(fwht128_quant_kernel<uint16_t, true>, (unsigned)((M * (H / 128) + 7) / 8), 256u, st, x, M,
+                        (int64_t)H, w.xq, w.sxg);
+    if (rc != W8A8_OK) return rc;
+    const int64_t nb = (M + bn - 1) / bn;
+    MoeSwapArgs a1 = {};
+    a1.counts = w.counts;
+    a1.offsets = w.offsets;
+    a1.tile_off = w.tile_off;
+    a1.E = 1;
+    a1.rows = 2 * I;
+    a1.K = H;
+    a1.ngroups = (2 * I) / 128;
+    a1.nkb = H / 128;
+    a1.a_out = w.a;
+    a1.early_plan = 1;   // the plan comes two kernels back
+    a1.gsx = w.sxg;
+    a1.gsw_u8 = u13;     // gate_up in the trunk's two-level format
+    a1.gsw_row = r13;
+    MoeSwapArgs a2 = a1;
+    a2.rows = H;
+    a2.K = I;
+    a2.ngroups = H / 128;
+    a2.nkb = I / 128;
+    a2.gsx = w.sag;
+    a2.gsw = s2;         // down on the group-128 grid
+    a2.gsw_u8 = nullptr;
+    a2.gsw_row = nullptr;
+    a2.row_tok = w.row_tok;
+    a2.row_slot = w.row_slot;
+    a2.row_w = w.row_w;
+    a2.contrib = w.out;
+    a2.topk = 1;
+    rc = bn == 16 ? launch_moe_swap<16, true, true>(w13, w.xq, M, a1, nb, st)
+       : bn == 32 ? launch_moe_swap<32, true, true>(w13, w.xq, M, a1, nb, st)
+                  : launch_moe_swap<64, true, true>(w13, w.xq, M, a1, nb, st);
+    if (rc != W8A8_OK) return rc;
+    rc = launch_chained(fwht128_quant_kernel<float, true>, (unsigned)((M * (I / 128) + 7) / 8), 256u, st,
+                        (const float*)w.a, M, (int64_t)I, w.qa, w.sag);
+    if (rc != W8A8_OK) return rc;
+    rc = bn == 16 ? launch_moe_swap<16, false, true>(w2, w.qa, M, a2, nb, st)
+       : bn == 32 ? launch_moe_swap<32, false, true>(w2, w.qa, M, a2, nb, st)
+                  : launch_moe_swap<64, false, true>(w2, w.qa, M, a2, nb, st);
+    if (rc != W8A8_OK) return rc;
+    rc = launch_chained(moe_finalize_kernel, (unsigned)((M * H / 4 + 255) / 256), 256u, st, (const float*)w.out, y,
+                        M, H, 1);
+    if (rc != W8A8_OK) return rc;
+    if (dbg) {
+        if (dbg->qx && cudaMemcpyAsync(dbg->qx, w.xq, (size_t)(M * H), cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->sx && cudaMemcpyAsync(dbg->sx, w.sxg, (size_t)M * (H / 128) * 2, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->qa && cudaMemcpyAsync(dbg->qa, w.qa, (size_t)M * I, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->sa && cudaMemcpyAsync(dbg->sa, w.sag, (size_t)M * (I / 128) * 2, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+    }
+    return W8A8_OK;
+}
+
+int w8a8_linear_trunk(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint8_t* su8, const uint16_t* s2,
+                      uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!su8 || !s2) return W8A8_ERR_INVALID_ARG;
+    return linear_group_scaled(qx, sx, qw, nullptr, y, M, N, K, 0.0078125f, (cudaStream_t)stream, su8, s2);
 }
 
 // ----------------------------------------------------------------- diagnostics

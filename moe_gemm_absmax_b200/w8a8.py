@@ -25,7 +25,8 @@ EXPORTS = (
     "w8a8_linear_noalloc_scratch_size", "w8a8_linear_noalloc",
     "w8a8_gemm_workspace_size", "w8a8_gemm_q", "w8a8_gemm_s32", "w8a8_moe_workspace_size",
     "w8a8_moe_forward", "w8a8_moe_g128_workspace_size", "w8a8_moe_g128_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
-    "group128_quant", "w8a8_linear_group128",
+    "group128_quant", "w8a8_linear_group128", "w8a8_trunk_weight_quant", "w8a8_linear_trunk",
+    "w8a8_shared_expert_workspace_size", "w8a8_shared_expert_forward",
     "w8a8_exp_proj",
     "w8a8_get_device_error", "w8a8_debug_wait_timeout", "w8a8_status_str", "w8a8_version",
 )
@@ -43,6 +44,10 @@ class MoeG128Debug(ctypes.Structure):
     _fields_ = [("topk_ids", ctypes.c_void_p), ("topk_w", ctypes.c_void_p), ("counts", ctypes.c_void_p),
                 ("qx", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("qa", ctypes.c_void_p),
                 ("sa", ctypes.c_void_p)]
+
+
+class SharedExpertDebug(ctypes.Structure):
+    _fields_ = [("qx", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("qa", ctypes.c_void_p), ("sa", ctypes.c_void_p)]
 
 
 class MlpDebug(ctypes.Structure):
@@ -86,6 +91,11 @@ def lib() -> ctypes.CDLL:
         "w8a8_linear_g128": ([vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "group128_quant": ([vp, i64, i64, vp, vp, vp], i32),
         "w8a8_linear_group128": ([vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
+        "w8a8_trunk_weight_quant": ([vp, i64, i64, vp, vp, vp, vp], i32),
+        "w8a8_linear_trunk": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
+        "w8a8_shared_expert_workspace_size": ([i64, i32, i32], sz),
+        "w8a8_shared_expert_forward": ([vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, vp, sz,
+                                        ctypes.POINTER(SharedExpertDebug), vp], i32),
         "w8a8_exp_proj": ([vp, vp, i64, vp], i32),
         "w8a8_get_device_error": ([vp, ctypes.POINTER(ctypes.c_int)], i32),
         "w8a8_debug_wait_timeout": ([i64, vp], i32),
@@ -415,6 +425,69 @@ def linear_group128(qx, sx, qw, sw, y=None, stream=None) -> torch.Tensor:
     _check(lib().w8a8_linear_group128(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(y), M, N, K, _stream(stream)),
            "w8a8_linear_group128")
     return y
+
+
+def trunk_weight_quant(w: torch.Tensor, stream=None):
+    """The trunk's two-level format of bf16 rows [N,K] (K % 256 == 0): returns
+    (codes int8 [N,K], u8 group scales [N,K/256], bf16 row scales [N])."""
+    _need(w, torch.bfloat16, "w", 2)
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    su8 = torch.empty((N, K // 256), dtype=torch.uint8, device=w.device)
+    s2 = torch.empty(N, dtype=torch.bfloat16, device=w.device)
+    _check(lib().w8a8_trunk_weight_quant(_ptr(w), N, K, _ptr(q), _ptr(su8), _ptr(s2), _stream(stream)),
+           "w8a8_trunk_weight_quant")
+    return q, su8, s2
+
+
+def linear_trunk(qx, sx, qw, su8, s2, y=None, stream=None) -> torch.Tensor:
+    """x codes + bf16 group scales (fwht128_quant) times W in the trunk format -> bf16 y [M,N]."""
+    _need(qx, torch.int8, "qx", 2)
+    _need(qw, torch.int8, "qw", 2)
+    _need(sx, torch.bfloat16, "sx", 2)
+    _need(su8, torch.uint8, "su8", 2)
+    _need(s2, torch.bfloat16, "s2", 1)
+    M, K = qx.shape
+    N = qw.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+    _check(lib().w8a8_linear_trunk(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(su8), _ptr(s2), _ptr(y), M, N, K,
+                                   _stream(stream)), "w8a8_linear_trunk")
+    return y
+
+
+def shared_expert_workspace_size(M: int, H: int, I: int) -> int:
+    return int(lib().w8a8_shared_expert_workspace_size(M, H, I))
+
+
+def shared_expert_forward(x, w13, u13, r13, w2, s2, y=None, ws=None, debug: bool = False, stream=None):
+    """The shared expert on the rotated grid: bf16 x [M,H]; gate_up in the trunk format
+    (w13 int8 [2I,H], u13 uint8 [2I,H/256], r13 bf16 [2I]); down on the group-128 grid
+    (w2 int8 [H,I], s2 bf16 [H,I/128]).  Returns y bf16 [M,H], or (y, debug dict)."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w13, torch.int8, "w13", 2)
+    _need(u13, torch.uint8, "u13", 2)
+    _need(r13, torch.bfloat16, "r13", 1)
+    _need(w2, torch.int8, "w2", 2)
+    _need(s2, torch.bfloat16, "s2", 2)
+    M, H = x.shape
+    I = w13.shape[0] // 2
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = _workspace(shared_expert_workspace_size(M, H, I), dev)
+    dbg_t = dbg_p = None
+    if debug:
+        dbg_t = dict(qx=torch.empty((M, H), dtype=torch.int8, device=dev),
+                     sx=torch.empty((M, H // 128), dtype=torch.bfloat16, device=dev),
+                     qa=torch.empty((M, I), dtype=torch.int8, device=dev),
+                     sa=torch.empty((M, I // 128), dtype=torch.bfloat16, device=dev))
+        dbg_p = ctypes.pointer(SharedExpertDebug(*[v.data_ptr() for v in dbg_t.values()]))
+    _check(lib().w8a8_shared_expert_forward(_ptr(x), _ptr(w13), _ptr(u13), _ptr(r13), _ptr(w2), _ptr(s2), _ptr(y),
+                                            M, H, I, _ptr(ws), ws.numel(), dbg_p, _stream(stream)),
+           "w8a8_shared_expert_forward")
+    return (y, dbg_t) if debug else y
 
 
 # ------------------------------------------------------------------ diagnostics
