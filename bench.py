@@ -573,6 +573,55 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         gbs = byts / (t * 1e-3) / 1e9
         out[f"head_group128_M{M}"] = {"ms": t, "gbs": gbs, "roofline": {"bound": "hbm", "frac": gbs / hbm, "peak": hbm,
                                                                          "unit": "GB/s", "bytes": byts}}
+    del qw, sw
+    # ---- trunk linear in the two-level format, on the Hadamard config's shapes (N = 4096, K = 2048)
+    d = inputs.HADAMARD
+    _, wb = inputs.hadamard_linear(0, 1)
+    tq, tu8, ts2 = w8a8.trunk_weight_quant(bf16_dev(torch, wb, dev))
+    for M in (1, 2048):
+        xb, _ = inputs.hadamard_linear(M, M)
+        x = bf16_dev(torch, xb, dev)
+        y = torch.empty((M, d["N"]), dtype=torch.bfloat16, device=dev)
+
+        def fn():
+            q, s = w8a8.fwht128_quant(x)
+            w8a8.linear_trunk(q, s, tq, tu8, ts2, y=y)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        N, K = tq.shape
+        ops = 2.0 * M * N * K
+        byts = N * K + N * (K // 256) + 2 * N + 2 * M * K + 2 * M * N
+        rec = {"ms": t, "tops": ops / (t * 1e-3) / 1e12, "gbs": byts / (t * 1e-3) / 1e9}
+        rec["roofline"] = ({"bound": "hbm", "frac": rec["gbs"] / hbm, "peak": hbm, "unit": "GB/s"} if M == 1 else
+                           {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"})
+        out[f"trunk_M{M}"] = rec
+    del tq, tu8, ts2
+    # ---- shared expert (gate_up in the trunk format, down on the group-128 grid), H = 2048, I = 512
+    H, I = inputs.MOE["H"], inputs.MOE["I"]
+    rng = np.random.default_rng([0, 3])
+    w13b = inputs.to_bf16_bits(inputs.weights(rng, (2 * I, H)))
+    w2b = inputs.to_bf16_bits(inputs.weights(rng, (H, I)))
+    sq13, su13, sr13 = w8a8.trunk_weight_quant(bf16_dev(torch, w13b, dev))
+    sq2, ss2 = w8a8.fwht128_quant(bf16_dev(torch, w2b, dev))
+    wbytes = sq13.numel() + su13.numel() + 2 * sr13.numel() + sq2.numel() + 2 * ss2.numel()
+    for M in (1, 8, 512, 4096):
+        xb, _ = inputs.moe_tokens(0, M)
+        x = bf16_dev(torch, xb, dev)
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.shared_expert_workspace_size(M, H, I), dtype=torch.uint8, device=dev)
+        fn = lambda: w8a8.shared_expert_forward(x, sq13, su13, sr13, sq2, ss2, y=y, ws=ws)
+        for _ in range(3):
+            fn()
+        t, _ = time_events(torch, fn, 10, flush=flush)
+        ops = 2.0 * M * 3 * H * I
+        byts = wbytes + 2 * M * H * 2
+        rec = {"ms": t, "tokens_per_s": M / (t * 1e-3), "tops": ops / (t * 1e-3) / 1e12,
+               "gbs": byts / (t * 1e-3) / 1e9}
+        rec["roofline"] = ({"bound": "hbm", "frac": rec["gbs"] / hbm, "peak": hbm, "unit": "GB/s"} if M <= 8 else
+                           {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"})
+        out[f"shared_expert_M{M}"] = rec
+        del x, y, ws
     return out
 
 
