@@ -88,29 +88,45 @@ __device__ __forceinline__ void fwht128_load4(const float* src, float (&v)[4]) {
     v[3] = raw.w;
 }
 
-// One warp per 128-wide block of a row; bf16 rows (activations, weights) or
+// Each warp quantizes kFwhtBlocksPerWarp consecutive 128-wide blocks (of one
+// row or of consecutive rows), all of their loads issued before the first
+// butterfly so that several are in flight; bf16 rows (activations, weights) or
 // fp32 rows (the routed experts' gated intermediate).  ROTATE = false is the
 // same group quantizer on the unrotated grid (the head's format: a bf16 scale
 // per row and 128 of K, no transform).  On a chain with programmatic
 // dependent launch it waits for the kernel before it (a no-op otherwise) and
 // reads its rows with coherent loads.
+constexpr int kFwhtBlocksPerWarp = 4;
+
 template <typename Tin, bool ROTATE = true>
 __global__ void __launch_bounds__(256) fwht128_quant_kernel(const Tin* __restrict__ x, int64_t M, int64_t K,
                                                             int8_t* __restrict__ q, uint16_t* __restrict__ s) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31;
-    const int64_t G = K / 128;
-    const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (blk >= M * G) return;
-    const int64_t m = blk / G, g = blk % G;
-    float v[4];
-    fwht128_load4(x + m * K + g * 128 + 4 * lane, v);
-    if constexpr (ROTATE) fwht128_warp(v, lane);
-    uint16_t sb;
-    const uint32_t pk = fwht128_codes(v, sb);
-    *reinterpret_cast<uint32_t*>(q + m * K + g * 128 + 4 * lane) = pk;
-    if (lane == 0) s[m * G + g] = sb;
+    const int64_t G = K / 128, nblk = M * G;
+    const int64_t blk0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kFwhtBlocksPerWarp;
+    if (blk0 >= nblk) return;
+    // block b of row m starts at m * K + g * 128 = b * 128: the blocks are contiguous
+    float v[kFwhtBlocksPerWarp][4];
+#pragma unroll
+    for (int i = 0; i < kFwhtBlocksPerWarp; ++i)
+        if (blk0 + i < nblk) fwht128_load4(x + (blk0 + i) * 128 + 4 * lane, v[i]);
+#pragma unroll
+    for (int i = 0; i < kFwhtBlocksPerWarp; ++i) {
+        if (blk0 + i >= nblk) break;
+        if constexpr (ROTATE) fwht128_warp(v[i], lane);
+        uint16_t sb;
+        const uint32_t pk = fwht128_codes(v[i], sb);
+        *reinterpret_cast<uint32_t*>(q + (blk0 + i) * 128 + 4 * lane) = pk;
+        if (lane == 0) s[blk0 + i] = sb;
+    }
+}
+
+// Grid of fwht128_quant_kernel for M rows of K (8 warps per CTA).
+inline int64_t fwht128_quant_ctas(int64_t M, int64_t K) {
+    const int64_t warps = (M * (K / 128) + kFwhtBlocksPerWarp - 1) / kFwhtBlocksPerWarp;
+    return (warps + 7) / 8;
 }
 
 constexpr int kG128MaxGroups = 64;

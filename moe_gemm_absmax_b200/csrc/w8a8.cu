@@ -1114,9 +1114,8 @@ int w8a8_moe_g128_forward(const uint16_t* x, const uint16_t* logits, const int8_
                   : launch_moe_swap<64, true, true>(w13, w.xq, R, a1, nb_max, st);
     if (rc != W8A8_OK) return rc;
     // the intermediate rotated along I and group-quantized
-    const int64_t blocks = R * (I / 128);
-    rc = launch_chained(fwht128_quant_kernel<float>, (unsigned)((blocks + 7) / 8), 256u, st, (const float*)w.a, R,
-                        (int64_t)I, w.qa, w.sag);
+    rc = launch_chained(fwht128_quant_kernel<float>, (unsigned)fwht128_quant_ctas(R, I), 256u, st, (const float*)w.a,
+                        R, (int64_t)I, w.qa, w.sag);
     if (rc != W8A8_OK) return rc;
     rc = bn == 16 ? launch_moe_swap<16, false, true>(w2, w.qa, R, a2, nb_max, st)
        : bn == 32 ? launch_moe_swap<32, false, true>(w2, w.qa, R, a2, nb_max, st)
@@ -1177,8 +1176,7 @@ int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, 
 int group_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, bool rotate, cudaStream_t st) {
     if (!x || !q || !s || M <= 0 || K <= 0 || K % 128 != 0) return W8A8_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 2)) return W8A8_ERR_INVALID_ARG;
-    const int64_t blocks = M * (K / 128);
-    const int64_t ctas = (blocks + 7) / 8;
+    const int64_t ctas = fwht128_quant_ctas(M, K);
     if (ctas > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
     if (rotate)
         fwht128_quant_kernel<uint16_t, true><<<(unsigned)ctas, 256, 0, st>>>(x, M, K, q, s);
@@ -1289,7 +1287,7 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
                                                                      w.row_tok, w.row_slot, w.row_w);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
     // x rotated along H and group-quantized: the sorted rows are the tokens
-    rc = launch_chained(fwht128_quant_kernel<uint16_t, true>, (unsigned)((M * (H / 128) + 7) / 8), 256u, st, x, M,
+    rc = launch_chained(fwht128_quant_kernel<uint16_t, true>, (unsigned)fwht128_quant_ctas(M, H), 256u, st, x, M,
                         (int64_t)H, w.xq, w.sxg);
     if (rc != W8A8_OK) return rc;
     const int64_t nb = (M + bn - 1) / bn;
@@ -1325,7 +1323,7 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
        : bn == 32 ? launch_moe_swap<32, true, true>(w13, w.xq, M, a1, nb, st)
                   : launch_moe_swap<64, true, true>(w13, w.xq, M, a1, nb, st);
     if (rc != W8A8_OK) return rc;
-    rc = launch_chained(fwht128_quant_kernel<float, true>, (unsigned)((M * (I / 128) + 7) / 8), 256u, st,
+    rc = launch_chained(fwht128_quant_kernel<float, true>, (unsigned)fwht128_quant_ctas(M, I), 256u, st,
                         (const float*)w.a, M, (int64_t)I, w.qa, w.sag);
     if (rc != W8A8_OK) return rc;
     rc = bn == 16 ? launch_moe_swap<16, false, true>(w2, w.qa, M, a2, nb, st)
