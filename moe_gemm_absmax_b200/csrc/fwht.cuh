@@ -88,32 +88,31 @@ __device__ __forceinline__ void fwht128_load4(const float* src, float (&v)[4]) {
     v[3] = raw.w;
 }
 
-// Each warp quantizes kFwhtBlocksPerWarp consecutive 128-wide blocks (of one
-// row or of consecutive rows), all of their loads issued before the first
-// butterfly so that several are in flight; bf16 rows (activations, weights) or
+// Each warp quantizes BPW consecutive 128-wide blocks (of one row or of
+// consecutive rows), all of their loads issued before the first butterfly so
+// that several are in flight (BPW = 4 for large inputs, 1 for a few rows,
+// where spreading the blocks over more warps is shorter); bf16 rows (activations, weights) or
 // fp32 rows (the routed experts' gated intermediate).  ROTATE = false is the
 // same group quantizer on the unrotated grid (the head's format: a bf16 scale
 // per row and 128 of K, no transform).  On a chain with programmatic
 // dependent launch it waits for the kernel before it (a no-op otherwise) and
 // reads its rows with coherent loads.
-constexpr int kFwhtBlocksPerWarp = 4;
-
-template <typename Tin, bool ROTATE = true>
+template <typename Tin, bool ROTATE = true, int BPW = 1>
 __global__ void __launch_bounds__(256) fwht128_quant_kernel(const Tin* __restrict__ x, int64_t M, int64_t K,
                                                             int8_t* __restrict__ q, uint16_t* __restrict__ s) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31;
     const int64_t G = K / 128, nblk = M * G;
-    const int64_t blk0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kFwhtBlocksPerWarp;
+    const int64_t blk0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * BPW;
     if (blk0 >= nblk) return;
     // block b of row m starts at m * K + g * 128 = b * 128: the blocks are contiguous
-    float v[kFwhtBlocksPerWarp][4];
+    float v[BPW][4];
 #pragma unroll
-    for (int i = 0; i < kFwhtBlocksPerWarp; ++i)
+    for (int i = 0; i < BPW; ++i)
         if (blk0 + i < nblk) fwht128_load4(x + (blk0 + i) * 128 + 4 * lane, v[i]);
 #pragma unroll
-    for (int i = 0; i < kFwhtBlocksPerWarp; ++i) {
+    for (int i = 0; i < BPW; ++i) {
         if (blk0 + i >= nblk) break;
         if constexpr (ROTATE) fwht128_warp(v[i], lane);
         uint16_t sb;
@@ -123,10 +122,31 @@ __global__ void __launch_bounds__(256) fwht128_quant_kernel(const Tin* __restric
     }
 }
 
-// Grid of fwht128_quant_kernel for M rows of K (8 warps per CTA).
+// Blocks per warp for M rows of K, and the grid (8 warps per CTA).
+inline int fwht128_quant_bpw(int64_t M, int64_t K) { return M * (K / 128) >= 148 * 8 * 8 ? 4 : 1; }
 inline int64_t fwht128_quant_ctas(int64_t M, int64_t K) {
-    const int64_t warps = (M * (K / 128) + kFwhtBlocksPerWarp - 1) / kFwhtBlocksPerWarp;
+    const int bpw = fwht128_quant_bpw(M, K);
+    const int64_t warps = (M * (K / 128) + bpw - 1) / bpw;
     return (warps + 7) / 8;
+}
+
+// Launches fwht128_quant_kernel (optionally chained with programmatic
+// dependent launch) with the block count per warp chosen for the size.
+template <typename Tin, bool ROTATE>
+cudaError_t launch_fwht128_quant(const Tin* x, int64_t M, int64_t K, int8_t* q, uint16_t* s, cudaStream_t st,
+                                 bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)fwht128_quant_ctas(M, K), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (fwht128_quant_bpw(M, K) == 4)
+        return cudaLaunchKernelEx(&cfg, fwht128_quant_kernel<Tin, ROTATE, 4>, x, M, K, q, s);
+    return cudaLaunchKernelEx(&cfg, fwht128_quant_kernel<Tin, ROTATE, 1>, x, M, K, q, s);
 }
 
 constexpr int kG128MaxGroups = 64;

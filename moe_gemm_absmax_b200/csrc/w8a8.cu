@@ -1114,8 +1114,7 @@ int w8a8_moe_g128_forward(const uint16_t* x, const uint16_t* logits, const int8_
                   : launch_moe_swap<64, true, true>(w13, w.xq, R, a1, nb_max, st);
     if (rc != W8A8_OK) return rc;
     // the intermediate rotated along I and group-quantized
-    rc = launch_chained(fwht128_quant_kernel<float>, (unsigned)fwht128_quant_ctas(R, I), 256u, st, (const float*)w.a,
-                        R, (int64_t)I, w.qa, w.sag);
+    rc = cuda_status(launch_fwht128_quant<float, true>(w.a, R, (int64_t)I, w.qa, w.sag, st, true));
     if (rc != W8A8_OK) return rc;
     rc = bn == 16 ? launch_moe_swap<16, false, true>(w2, w.qa, R, a2, nb_max, st)
        : bn == 32 ? launch_moe_swap<32, false, true>(w2, w.qa, R, a2, nb_max, st)
@@ -1178,11 +1177,8 @@ int group_quant(const uint16_t* x, int64_t M, int64_t K, int8_t* q, uint16_t* s,
     if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 2)) return W8A8_ERR_INVALID_ARG;
     const int64_t ctas = fwht128_quant_ctas(M, K);
     if (ctas > 0x7fffffffLL) return W8A8_ERR_UNSUPPORTED;
-    if (rotate)
-        fwht128_quant_kernel<uint16_t, true><<<(unsigned)ctas, 256, 0, st>>>(x, M, K, q, s);
-    else
-        fwht128_quant_kernel<uint16_t, false><<<(unsigned)ctas, 256, 0, st>>>(x, M, K, q, s);
-    return last_launch_status();
+    return cuda_status(rotate ? launch_fwht128_quant<uint16_t, true>(x, M, K, q, s, st, false)
+                              : launch_fwht128_quant<uint16_t, false>(x, M, K, q, s, st, false));
 }
 }  // namespace
 
@@ -1287,8 +1283,7 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
                                                                      w.row_tok, w.row_slot, w.row_w);
     if ((rc = last_launch_status()) != W8A8_OK) return rc;
     // x rotated along H and group-quantized: the sorted rows are the tokens
-    rc = launch_chained(fwht128_quant_kernel<uint16_t, true>, (unsigned)fwht128_quant_ctas(M, H), 256u, st, x, M,
-                        (int64_t)H, w.xq, w.sxg);
+    rc = cuda_status(launch_fwht128_quant<uint16_t, true>(x, M, (int64_t)H, w.xq, w.sxg, st, true));
     if (rc != W8A8_OK) return rc;
     const int64_t nb = (M + bn - 1) / bn;
     MoeSwapArgs a1 = {};
@@ -1323,8 +1318,7 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
        : bn == 32 ? launch_moe_swap<32, true, true>(w13, w.xq, M, a1, nb, st)
                   : launch_moe_swap<64, true, true>(w13, w.xq, M, a1, nb, st);
     if (rc != W8A8_OK) return rc;
-    rc = launch_chained(fwht128_quant_kernel<float, true>, (unsigned)fwht128_quant_ctas(M, I), 256u, st,
-                        (const float*)w.a, M, (int64_t)I, w.qa, w.sag);
+    rc = cuda_status(launch_fwht128_quant<float, true>(w.a, M, (int64_t)I, w.qa, w.sag, st, true));
     if (rc != W8A8_OK) return rc;
     rc = bn == 16 ? launch_moe_swap<16, false, true>(w2, w.qa, M, a2, nb, st)
        : bn == 32 ? launch_moe_swap<32, false, true>(w2, w.qa, M, a2, nb, st)
