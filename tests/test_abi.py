@@ -63,3 +63,34 @@ def test_argument_checks_without_gpu(L):
                               None, None) == w8a8.ERR_WORKSPACE
     assert L.w8a8_gemm_q(fake, fake, fake, fake, fake, 4, 16, 64, 7, None, 0, None) == w8a8.ERR_INVALID_ARG
     assert L.w8a8_debug_wait_timeout(10, None) == w8a8.ERR_INVALID_ARG
+
+
+def test_rotated_grid_workspace_queries(L):
+    # the FWHT128-grid MoE keeps the slot contributions [T*k, H] fp32 for the exact combine
+    assert L.w8a8_moe_g128_workspace_size(4096, 256, 2048, 512, 8) >= 4096 * 8 * 2048 * 4
+    assert L.w8a8_moe_g128_workspace_size(0, 256, 2048, 512, 8) == 0
+    assert L.w8a8_shared_expert_workspace_size(8, 2048, 512) >= 8 * 2048 * 4 + 8 * 512 * 4
+    assert L.w8a8_shared_expert_workspace_size(8, 128, 512) == 0
+
+
+def test_rotated_grid_argument_checks_without_gpu(L):
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    # K not a multiple of 128 (group grid), or of 256 (trunk format)
+    assert L.group128_quant(fake, 2, 192, fake, fake, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_linear_group128(fake, fake, fake, fake, fake, 2, 16, 192, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_trunk_weight_quant(fake, 4, 384, fake, fake, fake, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_trunk_weight_quant(fake, 4, 16384, fake, fake, fake, None) == w8a8.ERR_UNSUPPORTED
+    assert L.w8a8_linear_trunk(fake, fake, fake, fake, fake, fake, 2, 16, 384, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_linear_trunk(fake, fake, fake, None, fake, fake, 2, 16, 512, None) == w8a8.ERR_INVALID_ARG
+    # routed experts on the grid: H or I off the 128 grid, topk > E, too small a workspace
+    assert L.w8a8_moe_g128_forward(fake, fake, fake, fake, fake, fake, fake, 4, 8, 192, 128, 2, fake, 1 << 30,
+                                   None, None) == w8a8.ERR_UNSUPPORTED
+    assert L.w8a8_moe_g128_forward(fake, fake, fake, fake, fake, fake, fake, 4, 8, 256, 128, 9, fake, 1 << 30,
+                                   None, None) == w8a8.ERR_INVALID_ARG
+    assert L.w8a8_moe_g128_forward(fake, fake, fake, fake, fake, fake, fake, 4, 8, 256, 128, 2, fake, 64,
+                                   None, None) == w8a8.ERR_WORKSPACE
+    assert L.w8a8_shared_expert_forward(fake, fake, fake, fake, fake, fake, fake, 4, 384, 128, fake, 1 << 30,
+                                        None, None) == w8a8.ERR_UNSUPPORTED
+    assert L.w8a8_shared_expert_forward(fake, fake, fake, fake, fake, fake, fake, 4, 256, 128, fake, 64,
+                                        None, None) == w8a8.ERR_WORKSPACE
