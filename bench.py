@@ -633,7 +633,7 @@ HEAD = dict(N=131072, K=2048)
 # --------------------------------------------------------------------------- profiling cases
 CASES = ("gemv_gateup_m8", "gemv_down_m8", "prefill_gateup_m512", "prefill_down_m512", "prefill_gateup_m4096",
          "prefill_down_m4096", "quant_m4096_k17408", "quant_m4096_k5120", "moe_t1", "moe_t8", "moe_t512",
-         "moe_t4096", "moe_g128_t1", "moe_g128_t8", "moe_g128_t512", "moe_g128_t4096", "head_m1", "head_m8", "hadamard_m1",
+         "moe_t4096", "moe_g128_t1", "moe_g128_t8", "moe_g128_t512", "moe_g128_t4096", "head_m1", "head_m8", "shared_m1", "shared_m4096", "hadamard_m1",
          "hadamard_m200", "hadamard_m2048")
 
 
@@ -693,6 +693,17 @@ def run_case(name, torch, dev, reps=4):
         torch.cuda.empty_cache()
         for _ in range(reps):
             w8a8.moe_g128_forward(x, lg, q13, s13, q2, s2, k, y=y, ws=ws)
+    elif kind == "shared":
+        M = int(rest[1:])
+        H, I = inputs.MOE["H"], inputs.MOE["I"]
+        q13, u13, r13 = w8a8.trunk_weight_quant(randn(2 * I, H, std=0.02).to(torch.bfloat16))
+        q2, s2 = w8a8.fwht128_quant(randn(H, I, std=0.02).to(torch.bfloat16))
+        x = randn(M, H).to(torch.bfloat16)
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8a8.shared_expert_workspace_size(M, H, I), dtype=torch.uint8, device=dev)
+        torch.cuda.empty_cache()
+        for _ in range(reps):
+            w8a8.shared_expert_forward(x, q13, u13, r13, q2, s2, y=y, ws=ws)
     elif kind == "head":
         M = int(rest[1:])
         qw, sw = w8a8.group128_quant(randn(HEAD["N"], HEAD["K"], std=0.02).to(torch.bfloat16))

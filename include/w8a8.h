@@ -257,6 +257,8 @@ W8A8_API int w8a8_linear_trunk(const int8_t* qx, const uint16_t* sx, const int8_
  * Steps: (qx, sx) = fwht128_quant(x); v = the trunk product of (qx, sx) with
  * w13 (fp32); a_i = SiLU(v_2i) * v_2i+1; (qa, sa) = FWHT128 group quant of the
  * fp32 row a (along I); y = bf16( the group-128 product of (qa, sa) with w2 ).
+ * M <= 8 runs group-128 GEMVs (the gated one over w13 writes a), larger M the
+ * swap-AB tcgen05 expert kernels.
  * Requires H % 256 == 0, H <= 4096, I % 128 == 0, I <= 2048; 16-byte aligned
  * x, w13, w2, y; 256-byte aligned ws; ws_bytes >=
  * w8a8_shared_expert_workspace_size(M, H, I).  `dbg` may be NULL. */

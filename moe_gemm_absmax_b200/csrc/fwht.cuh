@@ -154,13 +154,20 @@ constexpr int kG128MaxGroups = 64;
 // One CTA per 16 weight rows; 8 warps split the K groups; tokens <= 8.  The
 // scales of the CTA's rows and tokens are staged in shared memory first, so
 // that the serial per-group promotion of warp 0 reads no global memory.
+// GATED: rows 2i / 2i+1 are gate_i / up_i (both in one CTA's 16 rows) and the
+// output is a[m, i] = SiLU(v_2i) * v_2i+1 in fp32 (a_out [M, N/2]) instead of
+// bf16 y.  On a chain with programmatic dependent launch the weight scales
+// are staged before the wait and the token codes and scales read after it
+// with coherent loads (a no-op wait otherwise).
+template <bool GATED>
 __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict__ qx,
                                                         const uint16_t* __restrict__ sx,
                                                         const int8_t* __restrict__ qw,
                                                         const uint16_t* __restrict__ sw, uint16_t* __restrict__ y,
                                                         int M, int N, int K, float post,
                                                         const uint8_t* __restrict__ sw_u8,
-                                                        const uint16_t* __restrict__ sw_row) {
+                                                        const uint16_t* __restrict__ sw_row,
+                                                        float* __restrict__ a_out) {
     __shared__ int4 pg[kG128MaxGroups][32];
     __shared__ float s_sw[16][kG128MaxGroups];   // [row in CTA][group]
     __shared__ float s_sx[8][kG128MaxGroups];    // [token][group]
@@ -176,9 +183,11 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
                       : bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp));
         s_sw[r][grp] = v;
     }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     for (int i = threadIdx.x; i < 8 * G; i += blockDim.x) {
         const int m = i / G, grp = i - m * G;
-        s_sx[m][grp] = m < M ? bf16_bits_to_float(__ldg(sx + (int64_t)m * G + grp)) : 0.0f;
+        s_sx[m][grp] = m < M ? bf16_bits_to_float(__ldcg(sx + (int64_t)m * G + grp)) : 0.0f;
     }
     const int8_t* w0 = qw + (int64_t)(block * 16 + g8) * K + 16 * t;
     const int8_t* w1 = w0 + 8 * (int64_t)K;
@@ -195,7 +204,7 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             uint4 xb = make_uint4(0, 0, 0, 0);
-            if (tok_ok) xb = __ldg(reinterpret_cast<const uint4*>(xr + grp * 128 + u * 64));
+            if (tok_ok) xb = __ldca(reinterpret_cast<const uint4*>(xr + grp * 128 + u * 64));
             const uint32_t A1[4] = {wa[u].x, wb[u].x, wa[u].y, wb[u].y};
             const uint32_t B1[2] = {xb.x, xb.y};
             const uint32_t A2[4] = {wa[u].z, wb[u].z, wa[u].w, wb[u].w};
@@ -222,7 +231,14 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
     for (int j = 0; j < 4; ++j) {
         const int m = 2 * t + (j & 1);
         const int n = block * 16 + g8 + 8 * (j >> 1);
-        if (m < M && n < N) y[(int64_t)m * N + n] = float_to_bf16_bits(__fmul_rn(yv[j], post));
+        const float v = __fmul_rn(yv[j], post);
+        if constexpr (GATED) {
+            // rows 2i (even g8) and 2i+1 (odd g8) sit in lanes 4 apart
+            const float up = __shfl_xor_sync(0xffffffffu, v, 4);
+            if (m < M && n < N && !(g8 & 1)) a_out[(int64_t)m * (N / 2) + (n >> 1)] = __fmul_rn(silu_proj(v), up);
+        } else {
+            if (m < M && n < N) y[(int64_t)m * N + n] = float_to_bf16_bits(v);
+        }
     }
 }
 

@@ -1155,8 +1155,8 @@ int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, 
         return W8A8_ERR_INVALID_ARG;
     if (M <= 8) {
         if (K / 128 > kG128MaxGroups || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
-        gemv_g128_kernel<<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post, sw_u8,
-                                                             sw_row);
+        gemv_g128_kernel<false><<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post,
+                                                                    sw_u8, sw_row, nullptr);
         return last_launch_status();
     }
     TcParams p = {};
@@ -1278,6 +1278,35 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
     cudaStream_t st = (cudaStream_t)stream;
     SharedWs w = shared_carve(ws, M, H, I);
     int rc;
+    auto debug_copies = [&]() -> int {
+        if (!dbg) return W8A8_OK;
+        if (dbg->qx && cudaMemcpyAsync(dbg->qx, w.xq, (size_t)(M * H), cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->sx && cudaMemcpyAsync(dbg->sx, w.sxg, (size_t)M * (H / 128) * 2, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->qa && cudaMemcpyAsync(dbg->qa, w.qa, (size_t)M * I, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        if (dbg->sa && cudaMemcpyAsync(dbg->sa, w.sag, (size_t)M * (I / 128) * 2, cudaMemcpyDeviceToDevice, st))
+            return W8A8_ERR_CUDA;
+        return W8A8_OK;
+    };
+    if (M <= 8 && H / 128 <= kG128MaxGroups && I / 128 <= kG128MaxGroups) {
+        // decode sizes: x quant, the gated group-128 GEMV over w13 (16 rows per
+        // CTA), the intermediate's quant, the group-128 GEMV over w2 writing y
+        rc = cuda_status(launch_fwht128_quant<uint16_t, true>(x, M, (int64_t)H, w.xq, w.sxg, st, false));
+        if (rc != W8A8_OK) return rc;
+        rc = launch_chained(gemv_g128_kernel<true>, (unsigned)(2 * I / 16), 256u, st, (const int8_t*)w.xq,
+                            (const uint16_t*)w.sxg, w13, (const uint16_t*)nullptr, (uint16_t*)nullptr, (int)M, 2 * I, H,
+                            0.0078125f, u13, r13, w.a);
+        if (rc != W8A8_OK) return rc;
+        rc = cuda_status(launch_fwht128_quant<float, true>(w.a, M, (int64_t)I, w.qa, w.sag, st, true));
+        if (rc != W8A8_OK) return rc;
+        rc = launch_chained(gemv_g128_kernel<false>, (unsigned)(H / 16), 256u, st, (const int8_t*)w.qa,
+                            (const uint16_t*)w.sag, w2, s2, y, (int)M, H, I, 0.0078125f, (const uint8_t*)nullptr,
+                            (const uint16_t*)nullptr, (float*)nullptr);
+        if (rc != W8A8_OK) return rc;
+        return debug_copies();
+    }
     const int bn = M <= 12 ? 16 : (M <= 24 ? 32 : 64);
     shared_plan_kernel<<<(unsigned)((M + 255) / 256), 256, 0, st>>>((int)M, bn, w.counts, w.offsets, w.tile_off,
                                                                      w.row_tok, w.row_slot, w.row_w);
@@ -1327,17 +1356,7 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
     rc = launch_chained(moe_finalize_kernel, (unsigned)((M * H / 4 + 255) / 256), 256u, st, (const float*)w.out, y,
                         M, H, 1);
     if (rc != W8A8_OK) return rc;
-    if (dbg) {
-        if (dbg->qx && cudaMemcpyAsync(dbg->qx, w.xq, (size_t)(M * H), cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-        if (dbg->sx && cudaMemcpyAsync(dbg->sx, w.sxg, (size_t)M * (H / 128) * 2, cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-        if (dbg->qa && cudaMemcpyAsync(dbg->qa, w.qa, (size_t)M * I, cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-        if (dbg->sa && cudaMemcpyAsync(dbg->sa, w.sag, (size_t)M * (I / 128) * 2, cudaMemcpyDeviceToDevice, st))
-            return W8A8_ERR_CUDA;
-    }
-    return W8A8_OK;
+    return debug_copies();
 }
 
 int w8a8_linear_trunk(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint8_t* su8, const uint16_t* s2,
