@@ -151,6 +151,9 @@ cudaError_t launch_fwht128_quant(const Tin* x, int64_t M, int64_t K, int8_t* q, 
 
 constexpr int kG128MaxGroups = 64;
 
+// Dynamic shared memory of gemv_g128_kernel for K / 128 = G groups (<= 39 KB).
+inline size_t gemv_g128_smem(int G) { return (size_t)G * (32 * 16 + 16 * 4 + 8 * 4); }
+
 // One CTA per 16 weight rows; 8 warps split the K groups; tokens <= 8.  The
 // scales of the CTA's rows and tokens are staged in shared memory first, so
 // that the serial per-group promotion of warp 0 reads no global memory.
@@ -168,12 +171,15 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
                                                         const uint8_t* __restrict__ sw_u8,
                                                         const uint16_t* __restrict__ sw_row,
                                                         float* __restrict__ a_out) {
-    __shared__ int4 pg[kG128MaxGroups][32];
-    __shared__ float s_sw[16][kG128MaxGroups];   // [row in CTA][group]
-    __shared__ float s_sx[8][kG128MaxGroups];    // [token][group]
+    // shared memory sized by the group count (gemv_g128_smem), so that short
+    // rows leave room for more CTAs per SM
+    extern __shared__ int4 g128_smem[];
+    const int G = K / 128;
+    int4* pg = g128_smem;                                               // [G][32] int32 partials
+    float* s_sw = reinterpret_cast<float*>(g128_smem + G * 32);         // [16][G] row scales
+    float* s_sx = s_sw + 16 * G;                                        // [8][G] token scales
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t = lane & 3;
-    const int G = K / 128;
     const int block = blockIdx.x;
     for (int i = threadIdx.x; i < 16 * G; i += blockDim.x) {
         const int r = i / G, grp = i - r * G, n = block * 16 + r;
@@ -181,13 +187,13 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
         if (n < N)   // the two-level trunk format: u8 per 256 of K times a bf16 row scale (exact)
             v = sw_u8 ? __fmul_rn((float)__ldg(sw_u8 + (int64_t)n * (G / 2) + grp / 2), bf16_bits_to_float(__ldg(sw_row + n)))
                       : bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp));
-        s_sw[r][grp] = v;
+        s_sw[r * G + grp] = v;
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     for (int i = threadIdx.x; i < 8 * G; i += blockDim.x) {
         const int m = i / G, grp = i - m * G;
-        s_sx[m][grp] = m < M ? bf16_bits_to_float(__ldcg(sx + (int64_t)m * G + grp)) : 0.0f;
+        s_sx[m * G + grp] = m < M ? bf16_bits_to_float(__ldcg(sx + (int64_t)m * G + grp)) : 0.0f;
     }
     const int8_t* w0 = qw + (int64_t)(block * 16 + g8) * K + 16 * t;
     const int8_t* w1 = w0 + 8 * (int64_t)K;
@@ -212,19 +218,19 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
             mma_s8_16832(acc, A1, B1);
             mma_s8_16832(acc, A2, B2);
         }
-        pg[grp][lane] = make_int4(acc[0], acc[1], acc[2], acc[3]);
+        pg[grp * 32 + lane] = make_int4(acc[0], acc[1], acc[2], acc[3]);
     }
     __syncthreads();
     if (warp != 0) return;
     float yv[4] = {0.f, 0.f, 0.f, 0.f};
     for (int grp = 0; grp < G; ++grp) {
-        const int4 p = pg[grp][lane];
+        const int4 p = pg[grp * 32 + lane];
         const int pv[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = 2 * t + (j & 1);
             const int r = g8 + 8 * (j >> 1);
-            if (m < M) yv[j] = __fmaf_rn(__int2float_rn(pv[j]), __fmul_rn(s_sx[m][grp], s_sw[r][grp]), yv[j]);
+            if (m < M) yv[j] = __fmaf_rn(__int2float_rn(pv[j]), __fmul_rn(s_sx[m * G + grp], s_sw[r * G + grp]), yv[j]);
         }
     }
 #pragma unroll

@@ -115,6 +115,10 @@ __device__ __forceinline__ MsBlock ms_block(const int* sp, int E, int b, int BN)
     return k;
 }
 
+// Fetch into L2 without waiting (the next unit's weight scales, which come
+// from HBM the first time an expert row is touched).
+__device__ __forceinline__ void ms_prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 template <int NT>
 __device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 
@@ -343,6 +347,15 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
         auto fetch = [&](int u) {
             const int b = u / a.ngroups;
             const MsBlock k = ms_block(sp, a.E, b, BN);
+            {   // this thread's weight-row scales of unit u
+                const int64_t wr = (int64_t)k.e * a.rows + (u - b * a.ngroups) * kMsBM + quarter * 32 + lane;
+                if (a.gsw_u8) {
+                    ms_prefetch_l2(a.gsw_u8 + wr * (G / 2));
+                    ms_prefetch_l2(a.gsw_row + wr);
+                } else {
+                    ms_prefetch_l2(a.gsw + wr * G);
+                }
+            }
             const bool have = mm < k.valid;
             const uint16_t* src = a.gsx + (int64_t)(k.row0 + mm) * G;
 #pragma unroll
@@ -485,7 +498,14 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                 }
             }
         };
+        // this thread's weight-row scale of unit u, into L2 one unit ahead
+        auto prefetch_sw = [&](int u) {
+            const int b = u / a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            ms_prefetch_l2(a.sw + (int64_t)k.e * a.rows + (u - b * a.ngroups) * kMsBM + quarter * 32 + lane);
+        };
         if (et < BN && (int)blockIdx.x < nunits) fetch(blockIdx.x);
+        if ((int)blockIdx.x < nunits) prefetch_sw(blockIdx.x);
         for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const int b = u / a.ngroups, g = u - b * a.ngroups;
             const MsBlock k = ms_block(sp, a.E, b, BN);
@@ -499,6 +519,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                 }
                 if (u + (int)gridDim.x < nunits) fetch(u + gridDim.x);
             }
+            if (u + (int)gridDim.x < nunits) prefetch_sw(u + gridDim.x);
             ms_epi_sync<128>();   // also: every warp is done with this buffer's use two units ago
             buf ^= 1;
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) break;

@@ -547,6 +547,19 @@ int launch_moe_swap(const int8_t* W, const int8_t* X, int64_t R, MoeSwapArgs a, 
 
 // A plain kernel launch on the MoE chain, with programmatic dependent launch.
 template <typename... KArgs, typename... Args>
+int launch_chained_smem(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                        Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    pdl_config(cfg, at, true);
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, args...));
+}
+
+template <typename... KArgs, typename... Args>
 int launch_chained(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t st, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
@@ -1155,8 +1168,8 @@ int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, 
         return W8A8_ERR_INVALID_ARG;
     if (M <= 8) {
         if (K / 128 > kG128MaxGroups || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
-        gemv_g128_kernel<false><<<(unsigned)(N / 16), 256, 0, st>>>(qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post,
-                                                                    sw_u8, sw_row, nullptr);
+        gemv_g128_kernel<false><<<(unsigned)(N / 16), 256, gemv_g128_smem((int)(K / 128)), st>>>(
+            qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post, sw_u8, sw_row, nullptr);
         return last_launch_status();
     }
     TcParams p = {};
@@ -1295,13 +1308,15 @@ int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, const uint8
         // CTA), the intermediate's quant, the group-128 GEMV over w2 writing y
         rc = cuda_status(launch_fwht128_quant<uint16_t, true>(x, M, (int64_t)H, w.xq, w.sxg, st, false));
         if (rc != W8A8_OK) return rc;
-        rc = launch_chained(gemv_g128_kernel<true>, (unsigned)(2 * I / 16), 256u, st, (const int8_t*)w.xq,
+        rc = launch_chained_smem(gemv_g128_kernel<true>, (unsigned)(2 * I / 16), 256u, gemv_g128_smem(H / 128), st,
+                                 (const int8_t*)w.xq,
                             (const uint16_t*)w.sxg, w13, (const uint16_t*)nullptr, (uint16_t*)nullptr, (int)M, 2 * I, H,
                             0.0078125f, u13, r13, w.a);
         if (rc != W8A8_OK) return rc;
         rc = cuda_status(launch_fwht128_quant<float, true>(w.a, M, (int64_t)I, w.qa, w.sag, st, true));
         if (rc != W8A8_OK) return rc;
-        rc = launch_chained(gemv_g128_kernel<false>, (unsigned)(H / 16), 256u, st, (const int8_t*)w.qa,
+        rc = launch_chained_smem(gemv_g128_kernel<false>, (unsigned)(H / 16), 256u, gemv_g128_smem(I / 128), st,
+                                 (const int8_t*)w.qa,
                             (const uint16_t*)w.sag, w2, s2, y, (int)M, H, I, 0.0078125f, (const uint8_t*)nullptr,
                             (const uint16_t*)nullptr, (float*)nullptr);
         if (rc != W8A8_OK) return rc;
