@@ -29,9 +29,11 @@
 // the weight tiles of its first stages before it waits for the codes of the
 // kernel just before.
 //
-// Roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..5
-// epilogue (TMEM lane quarters); the group-128 form has 8 epilogue warps
-// (lane quarter x half of the token block's columns).  All waits are bounded.
+// Roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..9
+// epilogue: in the per-token form two groups of four (one warp per TMEM lane
+// quarter), each owning one of the two accumulators and taking every other
+// unit; in the group-128 form lane quarter x half of the token block's
+// columns.  All waits are bounded.
 #pragma once
 
 #include "common.cuh"
@@ -59,7 +61,7 @@ struct MsSmem {
     static constexpr int kPlanOff = kTiles + kBars + 16;
     static constexpr int kPlanInts = 3 * 260;
     static constexpr int kRowOff = kPlanOff + kPlanInts * 4;
-    static constexpr int kRowBytes = 2 * 3 * 64 * 4;
+    static constexpr int kRowBytes = 2 * 2 * 3 * 64 * 4;   // [epilogue group][buffer][3][64]
     // group-128: the token block's scales, [2 buffers][group][row] fp32
     static constexpr int kSxOff = (kRowOff + kRowBytes + 15) / 16 * 16;   // read as float4
     static constexpr int kSxBytes = G128 ? 2 * kMsMaxGroups * BN * 4 : 0;
@@ -122,9 +124,13 @@ __device__ __forceinline__ void ms_prefetch_l2(const void* p) { asm volatile("pr
 template <int NT>
 __device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 
-// Threads: producer warp, MMA warp, then 4 epilogue warps (8 for the group-128 form).
+// Named barrier of one epilogue group of 4 warps (ids 1 and 2).
+__device__ __forceinline__ void ms_group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+
+// Threads: producer warp, MMA warp, then 8 epilogue warps (two groups of four
+// for the per-token form, lane quarter x column half for the group-128 form).
 template <bool G128>
-constexpr int ms_threads() { return G128 ? 320 : 192; }
+constexpr int ms_threads() { return 320; }
 
 template <int BN, bool GATED, bool G128 = false>
 __global__ void __launch_bounds__(ms_threads<G128>(), 1)
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], G128 ? 256 : 128);
+            mbar_init(&tempty[b], 128 * (G128 ? 2 : 1));
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -477,10 +483,17 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
         }
     } else {
         // ---------------------------------------------------------- epilogue
+        // Two groups of four warps (one per TMEM lane quarter); group j owns
+        // accumulator j and takes every other unit of this CTA, so that one
+        // group's per-unit latency (row data, TMEM read, stores) overlaps the
+        // other's.
+        const int grp = (warp - 2) >> 2;
         const int quarter = warp & 3;
-        const int et = threadIdx.x - 64;   // 0 .. 127
-        float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff);   // [2][3][64]
-        int acc = 0, buf = 0;
+        const int et = (threadIdx.x - 64) & 127;   // 0 .. 127 within the group
+        float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff) + grp * 2 * 3 * 64;   // [2][3][64]
+        const int acc = grp;
+        const int ustep = 2 * (int)gridDim.x;
+        int buf = 0;
         uint32_t acc_phase = 0;
         // row data of a token block, one row per thread (et < BN): loaded one
         // unit ahead so that its latency hides behind the current unit
@@ -504,9 +517,10 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             const MsBlock k = ms_block(sp, a.E, b, BN);
             ms_prefetch_l2(a.sw + (int64_t)k.e * a.rows + (u - b * a.ngroups) * kMsBM + quarter * 32 + lane);
         };
-        if (et < BN && (int)blockIdx.x < nunits) fetch(blockIdx.x);
-        if ((int)blockIdx.x < nunits) prefetch_sw(blockIdx.x);
-        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const int u0 = (int)blockIdx.x + grp * (int)gridDim.x;
+        if (et < BN && u0 < nunits) fetch(u0);
+        if (u0 < nunits) prefetch_sw(u0);
+        for (int u = u0; u < nunits; u += ustep) {
             const int b = u / a.ngroups, g = u - b * a.ngroups;
             const MsBlock k = ms_block(sp, a.E, b, BN);
             float* rs = s_row + buf * 3 * 64;
@@ -517,10 +531,10 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                     rs[64 + et] = __int_as_float(have ? nx_dst : 0);
                     rs[128 + et] = have ? nx_w : 0.0f;
                 }
-                if (u + (int)gridDim.x < nunits) fetch(u + gridDim.x);
+                if (u + ustep < nunits) fetch(u + ustep);
             }
-            if (u + (int)gridDim.x < nunits) prefetch_sw(u + gridDim.x);
-            ms_epi_sync<128>();   // also: every warp is done with this buffer's use two units ago
+            if (u + ustep < nunits) prefetch_sw(u + ustep);
+            ms_group_sync(1 + grp);   // also: the group is done with this buffer's use two units ago
             buf ^= 1;
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) break;
             tc_fence_after();
@@ -536,20 +550,25 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
-            if (++acc == 2) {
-                acc = 0;
-                acc_phase ^= 1u;
-            }
+            acc_phase ^= 1u;
             const int n = g * kMsBM + quarter * 32 + lane;   // weight row of expert e
             const float swn = __ldg(a.sw + (int64_t)k.e * a.rows + n);
             if constexpr (GATED) {
+                // lanes 2i (gate_i) and 2i+1 (up_i) split the columns: the even
+                // lane finishes the first half, the odd lane the second
                 const int I = a.rows >> 1;
                 float* arow = a.a_out + (int64_t)k.row0 * I + (n >> 1);
+                const bool odd = lane & 1;
+                float val[BN];
 #pragma unroll
-                for (int m = 0; m < BN; ++m) {
-                    const float val = __fmul_rn(__fmul_rn(__int2float_rn(v[m]), rs[m]), swn);
-                    const float up = __shfl_xor_sync(0xffffffffu, val, 1);   // row n + 1 (odd lane)
-                    if (m < k.valid && !(lane & 1)) arow[(int64_t)m * I] = __fmul_rn(silu_proj(val), up);
+                for (int m = 0; m < BN; ++m) val[m] = __fmul_rn(__fmul_rn(__int2float_rn(v[m]), rs[m]), swn);
+#pragma unroll
+                for (int j = 0; j < BN / 2; ++j) {
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? val[j] : val[j + BN / 2], 1);
+                    const float gv = odd ? other : val[j];
+                    const float uv = odd ? val[j + BN / 2] : other;
+                    const int m = j + (odd ? BN / 2 : 0);
+                    if (m < k.valid) arow[(int64_t)m * I] = __fmul_rn(silu_proj(gv), uv);
                 }
             } else {
                 const int H = a.rows;
