@@ -151,6 +151,10 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // group-128 form with units of at most 4 groups (K <= 512) and token
+    // blocks of at most 32 rows: two epilogue groups of four warps take
+    // alternate units, each with its own 4 TMEM slots (see the epilogue)
+    const bool alt = G128 && BN <= 32 && a.nkb <= 4;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -158,7 +162,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128 * (G128 ? 2 : 1));
+            mbar_init(&tempty[b], (G128 && !alt) ? 256 : 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -242,11 +246,17 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             // one accumulator slot per k block (= group): every slot holds the
             // conversion bias when it is released, so the MMAs always accumulate
             // and a slot's first use waits for phase 0 like every later one
+            // alternate-units mode (units of at most 4 groups): unit i of this
+            // CTA uses slots 4 (i & 1) + kb, each slot once every other unit
             constexpr uint32_t idesc = idesc_i8(kMsBM, BN);
-            int stage = 0, slot = 0;
+            int stage = 0, slot = 0, i = 0;
             uint32_t phase = 0, sphase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x, ++i) {
+                if (alt) {
+                    slot = 4 * (i & 1);
+                    sphase = (uint32_t)(i >> 1) & 1u;
+                }
                 for (int kb = 0; kb < a.nkb; ++kb) {
                     if (!mbar_wait_bounded(&tempty[slot], sphase, abort_flag, (kKernelIdMoeSwap << 16) | 3)) {
                         ok = false;
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                         stage = 0;
                         phase ^= 1u;
                     }
-                    if (++slot == kMsSlots) {
+                    if (++slot == kMsSlots) {   // (never reached in the alternate-units mode)
                         slot = 0;
                         sphase ^= 1u;
                     }
@@ -319,6 +329,147 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             mbar_wait_bounded(mma_done, 0u, nullptr, (kKernelIdMoeSwap << 16) | 5, 100000000ull);
         }
     } else if constexpr (G128) {
+      bool done = false;
+      if constexpr (BN <= 32) {
+        if (alt) {
+        // ---------------------------------------------------------- epilogue, group-128, alternate units
+        // Units of at most 4 groups: two groups of four warps (one per TMEM
+        // lane quarter, all BN columns each) take alternate units; group j
+        // owns slots 4j .. 4j+3, one per k block of its unit.  The promotion
+        // is that of the column-split form below.
+        done = true;
+        const int grp = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int et = (threadIdx.x - 64) & 127;   // 0 .. 127 within the group
+        float* s_row = reinterpret_cast<float*>(smem + SM::kRowOff) + grp * 2 * 3 * 64;   // [2][3][64]
+        float* s_sxg = reinterpret_cast<float*>(smem + SM::kSxOff) + grp * 2 * 4 * BN;    // [2][4][BN]
+        const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
+        const int G = a.nkb;
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+#pragma unroll
+            for (int c = 0; c < BN; c += 8) tmem_st_32x32b_x8_fill(tq + (uint32_t)((4 * grp + sl) * BN + c), 0x4B400000u);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        for (int sl = 0; sl < 4; ++sl) mbar_arrive(&tempty[4 * grp + sl]);
+        // the token block's group scales (thread et: row mm of group g0), loaded one unit ahead
+        const int mm = et & (BN - 1), g0 = et / BN;   // g0 < 128 / BN: every group of G <= 4
+        float nx_g = 0.0f, nx_w = 0.0f;
+        int nx_dst = 0;
+        auto fetch = [&](int u) {
+            const int b = u / a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            {   // this thread's weight-row scales of unit u
+                const int64_t wr = (int64_t)k.e * a.rows + (u - b * a.ngroups) * kMsBM + quarter * 32 + lane;
+                if (a.gsw_u8) {
+                    ms_prefetch_l2(a.gsw_u8 + wr * (G / 2));
+                    ms_prefetch_l2(a.gsw_row + wr);
+                } else {
+                    ms_prefetch_l2(a.gsw + wr * G);
+                }
+            }
+            nx_g = (mm < k.valid && g0 < G) ? bf16_bits_to_float(__ldcg(a.gsx + (int64_t)(k.row0 + mm) * G + g0)) : 0.0f;
+            if constexpr (!GATED) {
+                if (et < k.valid) {
+                    const int r = k.row0 + et;
+                    nx_dst = __ldcg(a.row_tok + r) * a.topk + __ldcg(a.row_slot + r);
+                    nx_w = __ldcg(a.row_w + r);
+                }
+            }
+        };
+        const int u0 = (int)blockIdx.x + grp * (int)gridDim.x;
+        const int ustep = 2 * (int)gridDim.x;
+        if (u0 < nunits) fetch(u0);
+        int buf = 0;
+        uint32_t kphase = 0;
+        const uint64_t magic2 = 0x4B4000004B400000ull;
+        const uint64_t inv2 = f2_pack(0.0078125f, 0.0078125f);
+        for (int u = u0; u < nunits; u += ustep) {
+            const int b = u / a.ngroups, g = u - b * a.ngroups;
+            const MsBlock k = ms_block(sp, a.E, b, BN);
+            float* rs = s_row + buf * 3 * 64;
+            float* sxs = s_sxg + buf * 4 * BN;
+            if (g0 < G) sxs[g0 * BN + mm] = nx_g;
+            if constexpr (!GATED) {
+                if (et < BN) {
+                    const bool have = et < k.valid;
+                    rs[64 + et] = __int_as_float(have ? nx_dst : 0);
+                    rs[128 + et] = have ? nx_w : 0.0f;
+                }
+            }
+            if (u + ustep < nunits) fetch(u + ustep);
+            ms_group_sync(1 + grp);   // also: the group is done with this buffer's use two units ago
+            buf ^= 1;
+            const int n = g * kMsBM + quarter * 32 + lane;   // weight row of expert e
+            const int64_t wr = (int64_t)k.e * a.rows + n;
+            const uint16_t* swrow = a.gsw + wr * G;
+            const uint8_t* swu8 = a.gsw_u8 ? a.gsw_u8 + wr * (G / 2) : nullptr;
+            const float swr = a.gsw_u8 ? bf16_bits_to_float(__ldg(a.gsw_row + wr)) : 0.0f;
+            uint64_t y2[BN / 2];
+#pragma unroll
+            for (int i = 0; i < BN / 2; ++i) y2[i] = 0ull;
+            bool ok = true;
+            for (int kb = 0; kb < G; ++kb) {
+                const float swg = swu8 ? __fmul_rn((float)__ldg(swu8 + kb / 2), swr) : bf16_bits_to_float(__ldg(swrow + kb));
+                const int slot = 4 * grp + kb;
+                if (!mbar_wait_bounded(&tfull[slot], kphase, abort_flag, (kKernelIdMoeSwap << 16) | 6)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t sw2 = f2_pack(swg, swg);
+                const float* sxk = sxs + kb * BN;
+                const uint32_t ta = tq + (uint32_t)(slot * BN);
+                uint32_t r[BN];
+                if constexpr (BN == 16) tmem_ld_32x32b_x16(ta, r);
+                else tmem_ld_32x32b_x32(ta, r);
+                tc_wait_ld();
+#pragma unroll
+                for (int c = 0; c < BN; c += 8) tmem_st_32x32b_x8_fill(ta + (uint32_t)c, 0x4B400000u);
+#pragma unroll
+                for (int q = 0; q < BN / 4; ++q) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(sxk + 4 * q);
+                    const uint64_t sc01 = f2_mul(f2_pack(s4.x, s4.y), sw2);
+                    const uint64_t sc23 = f2_mul(f2_pack(s4.z, s4.w), sw2);
+                    const uint64_t p01 = f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
+                    const uint64_t p23 =
+                        f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
+                    y2[2 * q] = f2_fma(p01, sc01, y2[2 * q]);
+                    y2[2 * q + 1] = f2_fma(p23, sc23, y2[2 * q + 1]);
+                }
+                tc_wait_st();
+                tc_fence_before();
+                mbar_arrive(&tempty[slot]);   // the slot goes back to the MMA
+            }
+            if (!ok) break;
+            kphase ^= 1u;
+            float v[BN];
+#pragma unroll
+            for (int i = 0; i < BN / 2; ++i) f2_unpack(f2_mul(y2[i], inv2), v[2 * i], v[2 * i + 1]);
+            if constexpr (GATED) {
+                const int I = a.rows >> 1;
+                float* arow = a.a_out + (int64_t)k.row0 * I + (n >> 1);
+                const bool odd = lane & 1;
+#pragma unroll
+                for (int j = 0; j < BN / 2; ++j) {
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? v[j] : v[j + BN / 2], 1);
+                    const float gv = odd ? other : v[j];
+                    const float uv = odd ? v[j + BN / 2] : other;
+                    const int m = j + (odd ? BN / 2 : 0);
+                    if (m < k.valid) arow[(int64_t)m * I] = __fmul_rn(silu_proj(gv), uv);
+                }
+            } else {
+                const int H = a.rows;
+#pragma unroll
+                for (int m = 0; m < BN; ++m)
+                    if (m < k.valid)
+                        a.contrib[(int64_t)__float_as_int(rs[64 + m]) * H + n] = __fmul_rn(rs[128 + m], v[m]);
+            }
+        }
+        }
+      }
+      if (!done) {
         // ---------------------------------------------------------- epilogue, group-128
         // y[n, m] = sum over groups g ascending of fma(float(p_g), sx[m, g] * sw[n, g], y)
         // in fp32, then * 1/128: two token rows per instruction (f32x2).  Each
@@ -481,6 +632,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                         a.contrib[(int64_t)__float_as_int(rs[64 + c0 + m]) * H + n] = __fmul_rn(rs[128 + c0 + m], v[m]);
             }
         }
+      }
     } else {
         // ---------------------------------------------------------- epilogue
         // Two groups of four warps (one per TMEM lane quarter); group j owns
