@@ -29,17 +29,21 @@
 namespace w8a8 {
 
 constexpr int kTc2BM = 256;       // rows per pair tile (128 per CTA)
-constexpr int kTc2BN = 256;       // columns per tile (128 B rows per CTA)
-constexpr int kTc2Stages = 6;
 constexpr int kTc2Threads = 192;
 constexpr int kKernelIdGemmTc2 = 4;
 
+// BN columns per pair tile: each CTA holds BN / 2 rows of B (256 or 160).
+// As many stages as fit: at a few hundred tokens every pair streams its own
+// weight columns from HBM, and the bytes in flight per SM set the pace.
+template <int BN>
 struct Tc2Smem {
     static constexpr int kA = 128 * kTcBK;                   // 16 KB per stage
-    static constexpr int kB = 128 * kTcBK;                   // 16 KB per stage
-    static constexpr int kTiles = kTc2Stages * (kA + kB);
-    static constexpr int kBars = (2 * kTc2Stages + 2 + 2 + 1) * 8;
+    static constexpr int kB = (BN / 2) * kTcBK;              // 16 / 10 KB per stage (multiples of 1 KB)
+    static constexpr int kStages = BN == 256 ? 6 : 8;
+    static constexpr int kTiles = kStages * (kA + kB);
+    static constexpr int kBars = (2 * kStages + 2 + 2 + 1) * 8;
     static constexpr int kBytes = 1024 + kTiles + kBars + 16;
+    static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -93,20 +97,21 @@ __device__ __forceinline__ void tc2_commit_pair(uint64_t* bar) {
         : "memory");
 }
 
-template <int EPI>
+template <int EPI, int BN = 256>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
     static_assert(EPI == kEpiBf16 || EPI == kEpiS32 || EPI == kEpiMoeGated, "dense epilogues");
-    constexpr int kCols = 2 * kTc2BN;   // two accumulators of 256 columns
-    using SM = Tc2Smem;
+    static_assert(BN % 32 == 0 && (BN / 2) % 8 == 0 && BN <= 256, "pair tile width");
+    constexpr int kCols = 2 * BN <= 256 ? 256 : 512;   // two accumulators of BN columns (a power of two)
+    using SM = Tc2Smem<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kTc2Stages * SM::kA;
+    uint8_t* sB = smem + SM::kStages * SM::kA;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kTiles);
     uint64_t* full = bars;                      // leader only
-    uint64_t* empty = bars + kTc2Stages;        // both
-    uint64_t* tfull = empty + kTc2Stages;       // both
+    uint64_t* empty = bars + SM::kStages;        // both
+    uint64_t* tfull = empty + SM::kStages;       // both
     uint64_t* tempty = tfull + 2;               // leader only
     uint64_t* mma_done = tempty + 2;            // leader only
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -117,7 +122,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTc2Stages; ++s) {
+        for (int s = 0; s < SM::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -164,17 +169,17 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                     const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2u * (SM::kA + SM::kB));
                     tma_load_2d_pair(sA + stage * SM::kA, &tmA, fb, kb * kTcBK, mt * kTc2BM + (int)rank * 128);
-                    tma_load_2d_pair(sB + stage * SM::kB, &tmB, fb, kb * kTcBK, nt * kTc2BN + (int)rank * 128);
+                    tma_load_2d_pair(sB + stage * SM::kB, &tmB, fb, kb * kTcBK, nt * BN + (int)rank * (BN / 2));
                     issued |= 1u << stage;
                     last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kTc2Stages) {
+                    if (++stage == SM::kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             if (!ok && leader) {
-                for (int s = 0; s < kTc2Stages; ++s)
+                for (int s = 0; s < SM::kStages; ++s)
                     if (issued & (1u << s))
                         mbar_wait_bounded(&full[s], (last_phase >> s) & 1u, nullptr, (kKernelIdGemmTc2 << 16) | 2,
                                           100000000ull);
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
         if (leader && lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kTc2BM, kTc2BN);
+            constexpr uint32_t idesc = idesc_i8(kTc2BM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
@@ -193,7 +198,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTc2BN);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < p.num_k_blocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, (kKernelIdGemmTc2 << 16) | 4)) {
                         ok = false;
@@ -207,7 +212,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                         tc2_mma_i8(d_tmem, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
                                    (kb > 0 || kk > 0) ? 1u : 0u);
                     tc2_commit_pair(&empty[stage]);   // frees this stage in both CTAs
-                    if (++stage == kTc2Stages) {
+                    if (++stage == SM::kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -238,13 +243,13 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
             const bool row_ok = row < p.M;
             float sxr = 0.0f;
             if ((EPI == kEpiBf16 || EPI == kEpiMoeGated) && row_ok) sxr = __ldg(p.sx + row);
-            const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kTc2BN);
+            const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
-            for (int c = 0; c < kTc2BN; c += 32) {
+            for (int c = 0; c < BN; c += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tq + (uint32_t)c, r);
                 tc_wait_ld();
-                const int n0 = nt * kTc2BN + c;
+                const int n0 = nt * BN + c;
                 if (!row_ok || n0 >= p.N) continue;
                 if (EPI == kEpiBf16) {
                     uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;

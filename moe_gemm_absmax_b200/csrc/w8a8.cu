@@ -110,17 +110,18 @@ int launch_tc(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     return last_launch_status();
 }
 
-// Pair-tile GEMM (cta_group::2, 256 x 256 tiles over two SMs).
-template <int EPI>
-int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
-    auto kern = gemm_i8_tc2_kernel<EPI>;
+// Pair-tile GEMM (cta_group::2, 256 x BN tiles over two SMs).
+template <int EPI, int BN>
+int launch_tc2_bn(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
+    using SM = Tc2Smem<BN>;
+    auto kern = gemm_i8_tc2_kernel<EPI, BN>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
     static int max_clusters[kMaxDevices] = {0};
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kTc2Threads, 1, 1);
-    cfg.dynamicSmemBytes = Tc2Smem::kBytes;
+    cfg.dynamicSmemBytes = SM::kBytes;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -130,7 +131,7 @@ int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     if (max_clusters[dev] == 0) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Smem::kBytes) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) != cudaSuccess)
             return W8A8_ERR_CUDA;
         cfg.gridDim = dim3((unsigned)(2 * (device_sms(dev) / 2)), 1, 1);
         int n = 0;
@@ -139,14 +140,36 @@ int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     }
     CUtensorMap ta, tb;
     if (!make_tmap_i8(&ta, A, (uint64_t)p.M, (uint64_t)p.K, 128)) return W8A8_ERR_CUDA;
-    if (!make_tmap_i8(&tb, B, (uint64_t)p.N, (uint64_t)p.K, 128)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tb, B, (uint64_t)p.N, (uint64_t)p.K, BN / 2)) return W8A8_ERR_CUDA;
     p.num_m_tiles = (p.M + kTc2BM - 1) / kTc2BM;
-    p.num_n_tiles = (p.N + kTc2BN - 1) / kTc2BN;
+    p.num_n_tiles = (p.N + BN - 1) / BN;
     p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
     const int tiles = p.num_m_tiles * p.num_n_tiles;
     const int clusters = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
     cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, p));
+}
+
+// Pair-tile width: 256 columns, or 160 where the narrower tile's better
+// filled last wave outweighs its higher operand ingest per MAC.  Per 128-byte
+// k block a CTA spends about max(MMA, ingest) cycles: MMA ~2.78 cycles per
+// column (256 x BN x 128 int8 MACs over the pair), ingest (16 KB of A +
+// 64 B per column of B) at ~43 B per cycle (both measured on the 256 tile).
+int pick_tc2_bn(int64_t M, int64_t N, int clusters) {
+    const int64_t mt = (M + kTc2BM - 1) / kTc2BM;
+    auto cost = [&](int bn) {
+        const int64_t tiles = mt * ((N + bn - 1) / bn);
+        const int64_t waves = (tiles + clusters - 1) / clusters;
+        const double kblock = std::max(2.78 * bn, (16384.0 + 64.0 * bn) / 43.0);
+        return (double)waves * kblock;
+    };
+    return cost(160) < cost(256) ? 160 : 256;
+}
+
+template <int EPI>
+int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
+    return pick_tc2_bn(p.M, p.N, current_sms() / 2) == 160 ? launch_tc2_bn<EPI, 160>(A, B, p, st)
+                                                           : launch_tc2_bn<EPI, 256>(A, B, p, st);
 }
 
 // Tile width: the one with less work in its last wave (256 on ties).
