@@ -134,6 +134,21 @@ def recorded_traffic(profile="gemv_decode_gateup_m8.md"):
 
 
 # --------------------------------------------------------------------------- timing helpers
+def max_over_ranks(torch, value, world, device):
+    """The largest of the ranks' values, on every rank (the value itself when alone):
+    a multi-GPU time is the slowest rank's."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, bytes_per_rank, ms):
+    """Whole-job GB/s: every rank streams bytes_per_rank per step, in the slowest rank's ms."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 def time_events(torch, fn, iters, flush=None):
     """Mean device time of fn() per call in ms, CUDA events on the current stream,
     one event pair per call; optional L2 flush between calls (outside the events).
@@ -328,12 +343,8 @@ def run_ours(args, rank, world, torch, dev):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * weight_bytes / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(torch, e0.elapsed_time(e1) / args.steps, world, dev)
+    value = job_throughput(world, weight_bytes, ms)
 
     # ---- roofline of the dominant kernel: the gate_up GEMV alone (pre-quantized codes)
     qx, sx = w8a8.quant_act(xs["gate_up"])
