@@ -113,3 +113,15 @@ def test_moe_full_size(orc, full_experts, T):
     rng = np.random.default_rng(T)
     tokens = None if T <= 8 else np.unique(np.concatenate([rng.integers(0, T, 24), [0, T - 1]]))
     _compare(orc, xb, lb, gw, ow, 8, tokens)
+
+
+def test_moe_full_size_extreme_skew(orc, full_experts):
+    """Every token's logits favour the same 8 experts: 512 rows each for those
+    (many token blocks per expert on the swap-AB path), 0 for the other 248."""
+    gw, ow = full_experts
+    xb, lb = inputs.moe_tokens(5, 512)
+    lf = inputs.bf16_bits_to_f32(lb).copy()
+    lf[:, [3, 17, 64, 65, 128, 200, 254, 255]] += 8.0
+    lb = inputs.to_bf16_bits(lf)
+    tokens = np.unique(np.concatenate([np.random.default_rng(11).integers(0, 512, 20), [0, 511]]))
+    _compare(orc, xb, lb, gw, ow, 8, tokens)

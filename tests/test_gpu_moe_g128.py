@@ -116,3 +116,23 @@ def test_moe_g128_full_size(orc, full_experts, T):
     rng = np.random.default_rng(T)
     tokens = None if T <= 8 else np.unique(np.concatenate([rng.integers(0, T, 24), [0, T - 1]]))
     _compare(orc, xb, lb, gw, ow, 8, tokens)
+
+
+def test_moe_g128_full_size_extreme_skew(orc, full_experts):
+    """Every token's logits favour the same 8 experts: 512 rows each for those,
+    none for the rest."""
+    gw, ow = full_experts
+    xb, lb = inputs.moe_tokens(5, 512)
+    lf = inputs.bf16_bits_to_f32(lb).copy()
+    lf[:, [3, 17, 64, 65, 128, 200, 254, 255]] += 8.0
+    lb = inputs.to_bf16_bits(lf)
+    tokens = np.unique(np.concatenate([np.random.default_rng(11).integers(0, 512, 20), [0, 511]]))
+    _compare(orc, xb, lb, gw, ow, 8, tokens)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 1), (3, 2, 2), (16, 256, 8)])
+def test_moe_g128_degenerate_routing(orc, T, E, k):
+    """top-1 of 8, every expert of 2 selected, and 16 tokens over 256 experts."""
+    xb, lb, w13, w2 = _small(T * 5 + E, T, E, 256, 128)
+    gw, ow = _rotate_experts(orc, w13, w2)
+    _compare(orc, xb, lb, gw, ow, k, None)
