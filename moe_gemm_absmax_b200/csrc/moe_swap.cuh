@@ -151,10 +151,10 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // group-128 form with units of at most 4 groups (K <= 512) and token
-    // blocks of at most 32 rows: two epilogue groups of four warps take
-    // alternate units, each with its own 4 TMEM slots (see the epilogue)
-    const bool alt = G128 && BN <= 32 && a.nkb <= 4;
+    // group-128 form with units of at most 4 groups (K <= 512): two epilogue
+    // groups of four warps take alternate units, each with its own 4 TMEM
+    // slots (see the epilogue)
+    const bool alt = G128 && a.nkb <= 4;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -330,13 +330,13 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
         }
     } else if constexpr (G128) {
       bool done = false;
-      if constexpr (BN <= 32) {
+      {
         if (alt) {
         // ---------------------------------------------------------- epilogue, group-128, alternate units
         // Units of at most 4 groups: two groups of four warps (one per TMEM
-        // lane quarter, all BN columns each) take alternate units; group j
-        // owns slots 4j .. 4j+3, one per k block of its unit.  The promotion
-        // is that of the column-split form below.
+        // lane quarter, all BN columns each, read 32 at a time) take alternate
+        // units; group j owns slots 4j .. 4j+3, one per k block of its unit.
+        // The promotion is that of the column-split form below.
         done = true;
         const int grp = (warp - 2) >> 2;
         const int quarter = warp & 3;
@@ -353,9 +353,13 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
         tc_wait_st();
         tc_fence_before();
         for (int sl = 0; sl < 4; ++sl) mbar_arrive(&tempty[4 * grp + sl]);
-        // the token block's group scales (thread et: row mm of group g0), loaded one unit ahead
-        const int mm = et & (BN - 1), g0 = et / BN;   // g0 < 128 / BN: every group of G <= 4
-        float nx_g = 0.0f, nx_w = 0.0f;
+        // the token block's group scales (thread et: row mm of groups g0, g0 + 128 / BN, ...),
+        // loaded one unit ahead
+        constexpr int JA = (4 * BN + 127) / 128;
+        constexpr int kGStepA = 128 / BN;
+        const int mm = et & (BN - 1), g0 = et / BN;
+        float nx_g[JA];
+        float nx_w = 0.0f;
         int nx_dst = 0;
         auto fetch = [&](int u) {
             const int b = u / a.ngroups;
@@ -369,7 +373,11 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                     ms_prefetch_l2(a.gsw + wr * G);
                 }
             }
-            nx_g = (mm < k.valid && g0 < G) ? bf16_bits_to_float(__ldcg(a.gsx + (int64_t)(k.row0 + mm) * G + g0)) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < JA; ++j) {
+                const int gg = g0 + kGStepA * j;
+                nx_g[j] = (mm < k.valid && gg < G) ? bf16_bits_to_float(__ldcg(a.gsx + (int64_t)(k.row0 + mm) * G + gg)) : 0.0f;
+            }
             if constexpr (!GATED) {
                 if (et < k.valid) {
                     const int r = k.row0 + et;
@@ -390,7 +398,11 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             const MsBlock k = ms_block(sp, a.E, b, BN);
             float* rs = s_row + buf * 3 * 64;
             float* sxs = s_sxg + buf * 4 * BN;
-            if (g0 < G) sxs[g0 * BN + mm] = nx_g;
+#pragma unroll
+            for (int j = 0; j < JA; ++j) {
+                const int gg = g0 + kGStepA * j;
+                if (gg < G) sxs[gg * BN + mm] = nx_g[j];
+            }
             if constexpr (!GATED) {
                 if (et < BN) {
                     const bool have = et < k.valid;
@@ -421,22 +433,27 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                 const uint64_t sw2 = f2_pack(swg, swg);
                 const float* sxk = sxs + kb * BN;
                 const uint32_t ta = tq + (uint32_t)(slot * BN);
-                uint32_t r[BN];
-                if constexpr (BN == 16) tmem_ld_32x32b_x16(ta, r);
-                else tmem_ld_32x32b_x32(ta, r);
-                tc_wait_ld();
+                constexpr int CW = BN < 32 ? BN : 32;   // columns per TMEM read
 #pragma unroll
-                for (int c = 0; c < BN; c += 8) tmem_st_32x32b_x8_fill(ta + (uint32_t)c, 0x4B400000u);
+                for (int c0 = 0; c0 < BN; c0 += CW) {
+                    uint32_t r[CW];
+                    if constexpr (CW == 16) tmem_ld_32x32b_x16(ta + (uint32_t)c0, r);
+                    else tmem_ld_32x32b_x32(ta + (uint32_t)c0, r);
+                    tc_wait_ld();
 #pragma unroll
-                for (int q = 0; q < BN / 4; ++q) {
-                    const float4 s4 = *reinterpret_cast<const float4*>(sxk + 4 * q);
-                    const uint64_t sc01 = f2_mul(f2_pack(s4.x, s4.y), sw2);
-                    const uint64_t sc23 = f2_mul(f2_pack(s4.z, s4.w), sw2);
-                    const uint64_t p01 = f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
-                    const uint64_t p23 =
-                        f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
-                    y2[2 * q] = f2_fma(p01, sc01, y2[2 * q]);
-                    y2[2 * q + 1] = f2_fma(p23, sc23, y2[2 * q + 1]);
+                    for (int c = 0; c < CW; c += 8) tmem_st_32x32b_x8_fill(ta + (uint32_t)(c0 + c), 0x4B400000u);
+#pragma unroll
+                    for (int q = 0; q < CW / 4; ++q) {
+                        const float4 s4 = *reinterpret_cast<const float4*>(sxk + c0 + 4 * q);
+                        const uint64_t sc01 = f2_mul(f2_pack(s4.x, s4.y), sw2);
+                        const uint64_t sc23 = f2_mul(f2_pack(s4.z, s4.w), sw2);
+                        const uint64_t p01 =
+                            f2_sub(f2_pack(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])), magic2);
+                        const uint64_t p23 =
+                            f2_sub(f2_pack(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])), magic2);
+                        y2[c0 / 2 + 2 * q] = f2_fma(p01, sc01, y2[c0 / 2 + 2 * q]);
+                        y2[c0 / 2 + 2 * q + 1] = f2_fma(p23, sc23, y2[c0 / 2 + 2 * q + 1]);
+                    }
                 }
                 tc_wait_st();
                 tc_fence_before();
