@@ -329,15 +329,12 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
             mbar_wait_bounded(mma_done, 0u, nullptr, (kKernelIdMoeSwap << 16) | 5, 100000000ull);
         }
     } else if constexpr (G128) {
-      bool done = false;
-      {
-        if (alt) {
+      if (alt) {
         // ---------------------------------------------------------- epilogue, group-128, alternate units
         // Units of at most 4 groups: two groups of four warps (one per TMEM
         // lane quarter, all BN columns each, read 32 at a time) take alternate
         // units; group j owns slots 4j .. 4j+3, one per k block of its unit.
         // The promotion is that of the column-split form below.
-        done = true;
         const int grp = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int et = (threadIdx.x - 64) & 127;   // 0 .. 127 within the group
@@ -484,9 +481,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                         a.contrib[(int64_t)__float_as_int(rs[64 + m]) * H + n] = __fmul_rn(rs[128 + m], v[m]);
             }
         }
-        }
-      }
-      if (!done) {
+      } else {
         // ---------------------------------------------------------- epilogue, group-128
         // y[n, m] = sum over groups g ascending of fma(float(p_g), sx[m, g] * sw[n, g], y)
         // in fp32, then * 1/128: two token rows per instruction (f32x2).  Each
