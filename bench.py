@@ -637,7 +637,7 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
 
 
 # head-shaped GEMM on the unrotated group-128 grid: the pages give no vocabulary
-# size, so a round 131072 rows over the MoE layer's hidden size
+# size, so 131072 (2^17) rows over the MoE layer's hidden size
 HEAD = dict(N=131072, K=2048)
 
 
