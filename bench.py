@@ -636,8 +636,9 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
     return out
 
 
-# head-shaped GEMM on the unrotated group-128 grid: the pages give no vocabulary
-# size, so 131072 (2^17) rows over the MoE layer's hidden size
+# head-shaped GEMM on the unrotated group-128 grid: "Qwen3.6-35B-A3B IQ8R - radiance
+# container" gives no vocabulary size, so 131072 (2^17) rows over the MoE layer's
+# hidden size
 HEAD = dict(N=131072, K=2048)
 
 

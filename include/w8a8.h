@@ -90,7 +90,7 @@ W8A8_API int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, u
                 void* ws, size_t ws_bytes, void* stream);
 
 /* Dense W8A8 linear for callers that cannot allocate device memory.
- * No counterpart on the pages: an interface addition of this library.
+ * No counterpart in the cited sources: an interface addition of this library.
  * Some callers cannot call cudaMalloc where they run the layer (an allocator
  * locked during a step, a plugin host that only passes its input and output
  * buffers).  This entry point computes exactly what w8a8_linear computes, with

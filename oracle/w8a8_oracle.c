@@ -5,7 +5,7 @@
  * or call this file: only the tests, the smoke check and the benchmark's
  * CPU-baseline leg use it.  It shares no code with the CUDA library.
  *
- * Plain scalar C, written for a reader to check against the pages by eye.
+ * Plain scalar C, written for a reader to check against the sources below by eye.
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC.
  * OpenMP is used only to split independent output rows across threads;
  * the arithmetic of each row is unchanged by it.
@@ -18,7 +18,7 @@
  *   [QUARK] "Qwen3.6-27B-Quark-W8A8-INT8", sections "Quantization Scheme"
  *            and "Quantization Details".
  *
- * Floating point: the pages fix fp32 scales, int32 accumulation and bf16
+ * Floating point: the sources fix fp32 scales, int32 accumulation and bf16
  * outputs, so the arithmetic below is fp32 with one IEEE round-to-nearest
  * operation per C operator (fp contraction is off); fp64 copies are kept
  * only where a test needs an error bound.
