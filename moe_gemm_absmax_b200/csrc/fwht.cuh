@@ -159,9 +159,10 @@ inline size_t gemv_g128_smem(int G) { return (size_t)G * (32 * 16 + 16 * 4 + 8 *
 // that the serial per-group promotion of warp 0 reads no global memory.
 // GATED: rows 2i / 2i+1 are gate_i / up_i (both in one CTA's 16 rows) and the
 // output is a[m, i] = SiLU(v_2i) * v_2i+1 in fp32 (a_out [M, N/2]) instead of
-// bf16 y.  On a chain with programmatic dependent launch the weight scales
-// are staged before the wait and the token codes and scales read after it
-// with coherent loads (a no-op wait otherwise).
+// bf16 y.  Launched with programmatic dependent launch, a CTA only prefetches
+// its weight rows into L2 before the dependency wait (L2 is coherent with
+// whatever kernel before it may still be writing them) and reads everything
+// after it, with coherent loads (the wait is a no-op otherwise).
 template <bool GATED>
 __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict__ qx,
                                                         const uint16_t* __restrict__ sx,
@@ -181,16 +182,22 @@ __global__ void __launch_bounds__(256) gemv_g128_kernel(const int8_t* __restrict
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t = lane & 3;
     const int block = blockIdx.x;
+    {   // this CTA's 16 weight rows into L2, one 128-byte line per thread and pass
+        const int64_t base = (int64_t)block * 16 * K, bytes = (int64_t)min(16, N - block * 16) * K;
+        for (int64_t o = (int64_t)threadIdx.x * 128; o < bytes; o += (int64_t)blockDim.x * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(qw + base + o));
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     for (int i = threadIdx.x; i < 16 * G; i += blockDim.x) {
         const int r = i / G, grp = i - r * G, n = block * 16 + r;
         float v = 0.0f;
         if (n < N)   // the two-level trunk format: u8 per 256 of K times a bf16 row scale (exact)
-            v = sw_u8 ? __fmul_rn((float)__ldg(sw_u8 + (int64_t)n * (G / 2) + grp / 2), bf16_bits_to_float(__ldg(sw_row + n)))
-                      : bf16_bits_to_float(__ldg(sw + (int64_t)n * G + grp));
+            v = sw_u8 ? __fmul_rn((float)__ldcg(sw_u8 + (int64_t)n * (G / 2) + grp / 2),
+                                  bf16_bits_to_float(__ldcg(sw_row + n)))
+                      : bf16_bits_to_float(__ldcg(sw + (int64_t)n * G + grp));
         s_sw[r * G + grp] = v;
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
     for (int i = threadIdx.x; i < 8 * G; i += blockDim.x) {
         const int m = i / G, grp = i - m * G;
         s_sx[m * G + grp] = m < M ? bf16_bits_to_float(__ldcg(sx + (int64_t)m * G + grp)) : 0.0f;

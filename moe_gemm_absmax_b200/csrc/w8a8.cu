@@ -1191,9 +1191,10 @@ int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, 
         return W8A8_ERR_INVALID_ARG;
     if (M <= 8) {
         if (K / 128 > kG128MaxGroups || N % 16 != 0) return W8A8_ERR_UNSUPPORTED;
-        gemv_g128_kernel<false><<<(unsigned)(N / 16), 256, gemv_g128_smem((int)(K / 128)), st>>>(
-            qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post, sw_u8, sw_row, nullptr);
-        return last_launch_status();
+        // chained: the weight rows go to L2 while the activation quant before it runs
+        return launch_chained_smem(gemv_g128_kernel<false>, (unsigned)(N / 16), 256u, gemv_g128_smem((int)(K / 128)),
+                                   st, qx, sx, qw, sw, y, (int)M, (int)N, (int)K, post, sw_u8, sw_row,
+                                   (float*)nullptr);
     }
     TcParams p = {};
     p.M = (int)M;
