@@ -269,10 +269,10 @@ def run_reference(args, rank, world):
               f"{rows['down']} of 5120 down rows; GB/s of those weight bytes")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 scales, bf16 out",
-            "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": "decode-shaped dense W8A8 linears, M=8 (gate_up 5120->34816, "
-                                   "down 17408->5120), CPU oracle on a row sample"},
+                                   "down 17408->5120), CPU oracle on a row sample",
+                       "arithmetic": "int8 x int8 -> int32, fp32 scales, bf16 out"},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
@@ -403,9 +403,10 @@ def run_ours(args, rank, world, torch, dev):
     clk.__exit__(None, None, None)
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 scales, bf16 in/out", "data": "synthetic",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": "decode-shaped dense W8A8 linears, M=8 tokens: gate_up K=5120->N=34816 then "
                                    "down K=17408->N=5120 (per-token act quant + weight-streaming GEMV + dequant)",
+                       "arithmetic": "int8 x int8 -> int32, fp32 scales, bf16 in/out",
                        "tokens": M, "weight_bytes_per_step": weight_bytes, "algorithmic_bytes_per_step": step_bytes,
                        "l2": "inputs larger than L2: 267 MB of weights streamed per step vs 126 MB L2",
                        "parallelism": f"replicas x{world}"},
