@@ -13,11 +13,12 @@
  *   [QUARK] "Qwen3.6-27B-Quark-W8A8-INT8" -- "Quantization Scheme" and
  *            "Quantization Details" (per-channel symmetric weights, per-token
  *            symmetric dynamic activations).
- *   [IQ8R]  "Qwen3.6-35B-A3B IQ8R - radiance container" -- file table (codes
- *            -127..127, each 128 of K rotated by the unnormalised Hadamard, a
- *            bf16 scale per row and 128 of K; activations int8 under the same
- *            rotation) and the conversion recipe (transform=fwht128 group=128
- *            scale=bf16 clamp=sym).
+ *   [IQ8R]  "Qwen3.6-35B-A3B IQ8R - radiance container" -- file table (int8
+ *            codes in -127..127 after every 128-wide slice of K is turned by
+ *            the unnormalised Hadamard matrix, one bf16 scale for each row and
+ *            each 128-wide slice; the activations quantized the same way) and
+ *            the conversion recipe (transform=fwht128 group=128 scale=bf16
+ *            clamp=sym).
  *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless stated otherwise; the caller owns
@@ -207,8 +208,9 @@ W8A8_API int w8a8_linear_g128(const int8_t* qx, const uint16_t* sx, const int8_t
                      int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ---------------------------------------------------------------------------
- * The group-128 grid without the rotation -- [IQ8R] file table (Head: "the
- * lm_head int8 with a bf16 scale per row and 128") and recipe row
+ * The group-128 grid without the rotation -- [IQ8R] file table (Head row:
+ * the lm_head holds int8 codes with one bf16 scale per row and 128 elements
+ * of K, and no rotation is listed for it) and recipe row
  * output.weight (codes=i8 group=128 scale=bf16 clamp=sym, no transform).
  * group128_quant: fwht128_quant without the butterflies: for each 128-wide
  * block of each row of x bf16 [M, K] (K % 128 == 0): s = bf16_rne(max|x| /
@@ -222,10 +224,11 @@ W8A8_API int w8a8_linear_group128(const int8_t* qx, const uint16_t* sx, const in
                                   uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ---------------------------------------------------------------------------
- * The trunk linears' two-level format -- [IQ8R] file table (Trunk: int8
- * codes -127..127 "with a u8 scale per row and 256 of K under a bf16 scale a
- * row, each 128 of K rotated by the unnormalised Hadamard, round to nearest")
- * and recipe (codes=i8 group=256 scale=u8 scale2=bf16 block2=1x*
+ * The trunk linears' two-level format -- [IQ8R] file table (Trunk row:
+ * int8 codes in -127..127; each 256-wide slice of a row has a u8 scale, and
+ * the row as a whole a bf16 scale that multiplies it; the rows are turned
+ * 128 elements at a time by the unnormalised Hadamard matrix; rounding to
+ * nearest) and recipe (codes=i8 group=256 scale=u8 scale2=bf16 block2=1x*
  * transform=fwht128 clamp=sym rule=search).
  * w8a8_trunk_weight_quant (set-up): each row of w bf16 [N, K] (K % 256 == 0,
  * K <= 8192) rotated 128 at a time; scale2[n] = bf16_rne(max|w'| / (127*255));
@@ -245,8 +248,9 @@ W8A8_API int w8a8_linear_trunk(const int8_t* qx, const uint16_t* sx, const int8_
                                const uint16_t* s2, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ---------------------------------------------------------------------------
- * The shared expert -- [IQ8R] file table (Experts: "the shared expert
- * likewise (its gate/up projection as the trunk's linears)") and recipe rows
+ * The shared expert -- [IQ8R] file table (Experts row: the shared expert is
+ * stored like the routed ones, except that its gate/up projection takes the
+ * trunk linears' format) and recipe rows
  * ffn_gate_up_shexp (the trunk format above) and ffn_down_shexp (group=128
  * scale=bf16 transform=fwht128).  A dense gated MLP on the rotated grid:
  *   x    bf16 [M, H]
@@ -275,10 +279,11 @@ W8A8_API int w8a8_shared_expert_forward(const uint16_t* x, const int8_t* w13, co
                                         void* ws, size_t ws_bytes, const w8a8_shared_expert_debug* dbg, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Routed experts on the FWHT128 grid -- [IQ8R] file table (Experts: int8 on
- * the same rotated grid with a bf16 scale per row and 128 of K; Activations:
- * int8 under the same rotation, the routed experts reading the codes the
- * trunk's quantisers write) and recipe (ffn_gate_up_exps / ffn_down_exps:
+ * Routed experts on the FWHT128 grid -- [IQ8R] file table (Experts row: the
+ * routed experts are int8 codes on the rotated grid, one bf16 scale for each
+ * row and 128-wide slice of K; Activations row: the activations are
+ * quantized after the same rotation, and the routed experts take the codes
+ * that the trunk's activation quantizer produces) and recipe (ffn_gate_up_exps / ffn_down_exps:
  * group=128 scale=bf16 transform=fwht128).  The layer of w8a8_moe_forward
  * with each quantizer replaced by fwht128_quant and each expert GEMM by its
  * group-128 form:

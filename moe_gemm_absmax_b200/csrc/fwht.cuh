@@ -1,7 +1,8 @@
 // FWHT128-domain W8A8 (a12, a13) -- "Qwen3.6-35B-A3B IQ8R - radiance
-// container": file table (each 128 of K rotated by the unnormalised Hadamard;
-// int8 codes -127..127 with a bf16 scale per row and 128 of K; activations
-// int8 under the same rotation) and the recipe (transform=fwht128 group=128
+// container": file table (every 128-wide slice of K turned by the
+// unnormalised Hadamard matrix; int8 codes in -127..127 with one bf16 scale
+// for each row and slice; the activations quantized after the same
+// rotation) and the recipe (transform=fwht128 group=128
 // scale=bf16 clamp=sym).
 //
 // fwht128_warp / fwht128_quant_kernel: one warp per 128-wide block of a row.  Lane l holds

@@ -5,7 +5,7 @@
 //   acc[m,n] = sum_k A[m,k] B[n,k]                      A = codes [M,K], B = weights [N,K]
 //   y[m,n]   = bf16_rne( (float(acc) * sx[m]) * sw[n] )  (or the raw int32 acc)
 // (a13) group-128 scaled, rotated domain -- "Qwen3.6-35B-A3B IQ8R - radiance
-// container", file table (a bf16 scale per row and 128 of K):
+// container", file table (one bf16 scale for each row and 128-wide slice of K):
 //   p_g      = sum over the 128 k of group g of A[m,k] B[n,k]   (one TMEM tile per g)
 //   acc      = fma(float(p_g), float(sx[m,g]) * float(sw[n,g]), acc), g ascending
 //   y[m,n]   = bf16_rne(acc * (1/128))

@@ -1,7 +1,8 @@
 // Routed experts on the FWHT128 grid -- "Qwen3.6-35B-A3B IQ8R - radiance
-// container", file table (Experts: int8 on the same rotated grid with a bf16
-// scale per row and 128 of K; Activations: int8 under the same rotation, the
-// routed experts reading the codes the trunk's quantisers write) and the
+// container", file table (Experts row: int8 codes on the rotated grid with
+// one bf16 scale per row and 128-wide slice of K; Activations row: the
+// activations quantized after the same rotation, the routed experts taking
+// the codes of the trunk's activation quantizer) and the
 // recipe rows of the experts' gate_up and down weights (group=128 scale=bf16
 // transform=fwht128).
 //

@@ -533,8 +533,8 @@ void oracle_fwht128_quant_f32(const float* x, int64_t M, int64_t K, int8_t* q, b
 
 /* ------------------------------------------------------------------ */
 /* Group-128 quantization without the rotation (f3: [IQ8R] file table,  */
-/* Head: "the lm_head int8 with a bf16 scale per row and 128"; recipe    */
-/* row output.weight: codes=i8 group=128 scale=bf16 clamp=sym, no        */
+/* Head row: int8 codes, one bf16 scale per row and 128 of K, no         */
+/* rotation listed; recipe row output.weight: codes=i8 group=128 scale=bf16 clamp=sym, no        */
 /* transform).  Each 128-wide block of each row: s = bf16_rne(absmax /  */
 /* 127), codes from that stored scale -- the block quantizer above       */
 /* without the butterflies.                                              */
@@ -604,10 +604,10 @@ void oracle_gemm_group128(const int8_t* qx, const bf16_t* sx, const int8_t* qw, 
 }
 
 /* ------------------------------------------------------------------ */
-/* f4: the trunk linears' two-level scales ([IQ8R] file table, Trunk:    */
-/* int8 codes -127..127 "with a u8 scale per row and 256 of K under a    */
-/* bf16 scale a row, each 128 of K rotated by the unnormalised          */
-/* Hadamard, round to nearest"; recipe: codes=i8 group=256 scale=u8      */
+/* f4: the trunk linears' two-level scales ([IQ8R] file table, Trunk     */
+/* row: int8 codes in -127..127, a u8 scale for each row and 256-wide    */
+/* slice of K times a bf16 scale for the row, rows turned 128 at a time  */
+/* by the unnormalised Hadamard matrix, rounding to nearest; recipe: codes=i8 group=256 scale=u8      */
 /* scale2=bf16 block2=1x* transform=fwht128 clamp=sym rule=search).      */
 /* Per row n of W (bf16 [N, K], K % 256 == 0), after the rotation of     */
 /* each 128 of K:                                                         */
@@ -690,10 +690,11 @@ void oracle_gemm_trunk(const int8_t* qx, const bf16_t* sx, const int8_t* qw, con
 }
 
 /* ------------------------------------------------------------------ */
-/* f1: routed experts on the rotated grid ([IQ8R] file table: "Experts   */
-/* ... int8 on the same rotated grid with a bf16 scale per row and 128  */
-/* of K"; "Activations int8 under the same rotation, the routed experts  */
-/* reading the codes the trunk's quantisers write"; recipe rows          */
+/* f1: routed experts on the rotated grid ([IQ8R] file table, Experts    */
+/* row: int8 codes on the rotated grid with one bf16 scale per row and   */
+/* 128-wide slice of K; Activations row: activations quantized after the */
+/* same rotation, the routed experts taking the trunk quantizer's codes; */
+/* recipe rows                                                            */
 /* ffn_gate_up_exps / ffn_down_exps: group=128 scale=bf16                 */
 /* transform=fwht128).  The pipeline is that of oracle_moe_forward with  */
 /* each quantizer replaced by the FWHT128 group quantizer and each GEMM  */
@@ -785,8 +786,9 @@ void oracle_moe_g128_forward(const bf16_t* x, const bf16_t* logits,
 }
 
 /* ------------------------------------------------------------------ */
-/* f3: the shared expert ([IQ8R] file table, Experts: "the shared expert  */
-/* likewise (its gate/up projection as the trunk's linears)"; recipe rows */
+/* f3: the shared expert ([IQ8R] file table, Experts row: stored like the */
+/* routed experts, its gate/up projection in the trunk's format; recipe   */
+/* rows                                                                   */
 /* ffn_gate_up_shexp: the trunk's two-level format, ffn_down_shexp:       */
 /* group=128 scale=bf16 transform=fwht128).  A dense gated MLP on the     */
 /* rotated grid, for each token m:                                         */

@@ -50,7 +50,7 @@ def test_linear_g128(orc, M):
     assert exact == 1.0
 
 
-# ---- the unrotated group-128 grid (the head's format: a bf16 scale per row and 128, no transform)
+# ---- the unrotated group-128 grid (the head's format: one bf16 scale per row and 128 of K, no rotation)
 
 @pytest.mark.parametrize("M", [1, 3, 2048])
 def test_group128_quant_bit_exact(orc, M):

@@ -1,8 +1,8 @@
 """Pins of the oracle's FWHT128 group quantization (a12) and group-128
 scaled GEMM (a13): "Qwen3.6-35B-A3B IQ8R - radiance container", file table
-(Trunk: each 128 of K rotated by the unnormalised Hadamard; Experts: a bf16
-scale per row and 128 of K on the same rotated grid; Activations: int8 under
-the same rotation) and the conversion recipe (transform=fwht128 group=128
+(Trunk row: every 128-wide slice of K turned by the unnormalised Hadamard
+matrix; Experts row: one bf16 scale for each row and 128-wide slice on that
+rotated grid; Activations row: quantized after the same rotation) and the conversion recipe (transform=fwht128 group=128
 scale=bf16 clamp=sym).
 
 The transform is pinned to scipy's Sylvester Hadamard matrix (a library

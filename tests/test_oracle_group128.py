@@ -1,6 +1,6 @@
 """Pins of the oracle's group-128 grid without the rotation (the head's
-format: "Qwen3.6-35B-A3B IQ8R - radiance container", file table, Head: the
-lm_head int8 with a bf16 scale per row and 128 of K; recipe row
+format: "Qwen3.6-35B-A3B IQ8R - radiance container", file table, Head row:
+int8 codes with one bf16 scale per row and 128 of K, no rotation; recipe row
 output.weight: codes=i8 group=128 scale=bf16 clamp=sym, no transform).
 
 The quantizer is pinned by brute force (each code is the nearest of the 255

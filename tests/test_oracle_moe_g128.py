@@ -1,7 +1,8 @@
 """Pins of the oracle's routed experts on the FWHT128 grid: "Qwen3.6-35B-A3B
-IQ8R - radiance container", file table (Experts: int8 on the same rotated
-grid with a bf16 scale per row and 128 of K; Activations: int8 under the same
-rotation, the routed experts reading the codes the trunk's quantisers write)
+IQ8R - radiance container", file table (Experts row: int8 codes on the
+rotated grid, one bf16 scale per row and 128-wide slice of K; Activations
+row: quantized after the same rotation, the routed experts taking the trunk
+quantizer's codes)
 and the recipe rows of the routed experts' gate_up and down weights
 (group=128 scale=bf16 transform=fwht128).
 

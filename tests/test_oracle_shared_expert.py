@@ -1,6 +1,6 @@
 """Pins of the oracle's shared expert on the rotated grid ("Qwen3.6-35B-A3B
-IQ8R - radiance container", file table, Experts: the shared expert likewise,
-its gate/up projection as the trunk's linears; recipe rows ffn_gate_up_shexp
+IQ8R - radiance container", file table, Experts row: stored like the routed
+experts, with its gate/up projection in the trunk's format; recipe rows ffn_gate_up_shexp
 (two-level trunk format) and ffn_down_shexp (group=128 scale=bf16
 transform=fwht128)).
 
