@@ -18,8 +18,9 @@
 //     mma #1: A = {w0, v0, w1, v1}, B = {x0, x1};  mma #2: A = {w2, v2, w3, v3}, B = {x2, x3}
 //   and C = {(r0+g, 2t), (r0+g, 2t+1), (r0+g+8, 2t), (r0+g+8, 2t+1)} (token columns).
 //
-// A CTA (8 warps) owns WN blocks of 16 weight rows; WK warps split each
-// block's K range and meet in shared memory.  When gridDim.y > 1 the K range
+// A CTA (8 warps) owns WN blocks of 16 weight rows (WN = 4, 2 or 1); WK =
+// 8 / WN warps split each block's K range and meet in shared memory.  When
+// gridDim.y > 1 the K range
 // is also split over CTAs: each writes its int32 partial to the workspace
 // and the last CTA to arrive (counter per row block) adds them in order and
 // runs the epilogue -- integer sums, so the result is exact and
@@ -54,6 +55,7 @@ struct GemvShape {
     int nchunks;          // ceil(K / 64)
     int32_t* part;        // split-K partials [nkseg][row blocks][TG][32][4] (nkseg > 1)
     int* counters;        // arrival counters, one per CTA column, zero on entry (nkseg > 1)
+    int trig;             // let the next kernel on the stream launch at once (programmatic launch)
 };
 
 // Computes this warp's int32 C fragments over its K range and reduces them
@@ -67,6 +69,11 @@ __device__ __forceinline__ bool gemv_core(const GemvShape& a, int (&acc)[TG][4],
     static_assert(WN * WK == kGemvThreads / 32, "8 warps");
     __shared__ __align__(16) int red[WK > 1 ? WK - 1 : 1][WN][TG][32][4];   // read and written as int4
     __shared__ int is_last;
+    // A kernel launched after this one with programmatic serialization may
+    // start now: it waits for this grid's completion before it reads anything
+    // (the library's quant kernels, which come next in a decode chain, also
+    // hold their own dependents back until that wait returns).
+    if (a.trig) asm volatile("griddepcontrol.launch_dependents;");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wn = warp % WN, wk = warp / WN;

@@ -396,6 +396,7 @@ __global__ void __launch_bounds__(kGemvThreads) moe_gemm_kernel(MoeGemmArgs m) {
     a.nchunks = (m.K + 63) / 64;
     a.part = nullptr;
     a.counters = nullptr;
+    a.trig = 0;
     const float* swe = m.sw + (int64_t)e * m.rows;
     for (int tok0 = 0; tok0 < cnt; tok0 += 8 * TG) {
         a.x = m.xq + (int64_t)(off + tok0) * m.K;

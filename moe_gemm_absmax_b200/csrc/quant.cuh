@@ -115,6 +115,18 @@ __device__ __forceinline__ void quant_vec_store(const uint4& raw, const QuantRow
     store_codes<E>(dst, packed);
 }
 
+// Start of every quant kernel.  It may be launched to overlap the kernel
+// before it on the stream (programmatic dependent launch), so it touches no
+// memory before griddepcontrol.wait: x may come from that kernel, and q / s
+// may still be read by it.  Only after the wait does it let the kernel after
+// it launch (that kernel streams weights before its own wait), so that
+// everything before this quant kernel on the stream has completed by the
+// time anything after it runs.
+__device__ __forceinline__ void quant_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
 __device__ __forceinline__ void cp_async_16(void* smem, const void* gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
                  "l"(gmem)
@@ -133,8 +145,7 @@ __global__ void __launch_bounds__(NT) quant_rows_smem_kernel(const Tin* __restri
     using VT = VecTraits<Tin>;
     constexpr int E = VT::kElems;
     extern __shared__ __align__(16) uint4 row_s[];
-    asm volatile("griddepcontrol.launch_dependents;");
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // x may come from the kernel just before
+    quant_dependency_wait();
     const int64_t row = blockIdx.x;
     const int nvec = (int)(K / E);
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
@@ -171,10 +182,7 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const Tin* __restrict__ 
                                                         int8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
                                                         int vpc, int cl, int* zero_buf, int zero_n) {
     using VT = VecTraits<Tin>;
-    // let a kernel launched after this one with programmatic serialization
-    // start its independent prologue now (it still waits for our results)
-    asm volatile("griddepcontrol.launch_dependents;");
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // x may come from the kernel just before
+    quant_dependency_wait();
     // optional side job: clear a small int buffer that a later kernel on the
     // same stream expects to find zero (split-K arrival counters)
     for (int i = blockIdx.x * NT + threadIdx.x; i < zero_n; i += gridDim.x * NT) zero_buf[i] = 0;
@@ -246,8 +254,7 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const Tin* __restr
     using VT = VecTraits<Tin>;
     constexpr int E = VT::kElems;
     constexpr int kMaxV = 8;
-    asm volatile("griddepcontrol.launch_dependents;");
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // x may come from the kernel just before
+    quant_dependency_wait();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;

@@ -201,26 +201,35 @@ int run_tc(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw,
 
 // ----------------------------------------------------------------- GEMV
 // Decode GEMV.  M <= 8: the register-streaming mma.sync kernel
-// (gemv_dense_kernel): 4 row blocks x 2 K-halves per CTA, 4 chunks of
-// weight loads in flight per thread, 64 registers so that 4 CTAs (32 warps)
-// stay resident per SM, and the K range split over `nkseg` CTAs until the
-// CTAs fill about 70% of those slots (measured fastest for both decode
-// shapes: more splits cost more in partial sums than they gain).  9 <= M <= 32: the swap-AB tcgen05 kernel (gemv_tc_kernel),
-// whose token columns grow for free.  Plans are fixed per shape
-// (independent of the device) so that workspace sizes are too.
+// (gemv_dense_kernel): WN row blocks of 16 rows x WK = 8 / WN K-slices per
+// CTA, 4 chunks of weight loads in flight per thread, 64 registers so that
+// 4 CTAs (32 warps) stay resident per SM.  WN is the largest of 4, 2, 1 that
+// still gives at least half a wave of CTAs (296 on 148 SMs); only when even
+// 16-row CTAs do not reach that is the K range also split over `nkseg` CTAs
+// (partials in the workspace), until the CTAs fill about 70% of the slots.
+// The GEMV lets the next kernel launch at once when its own CTAs fill most
+// of the SM slots (the wide gate_up shapes); measured on the decode step of
+// the dense MLP shapes with two weight sets alternating (gate_up 4 x 2
+// warps, 544 CTAs, early launch; down 1 x 8 warps, 320 CTAs, no split, no
+// early launch: 54.1 us a step against 61.8 us for a 5-way split of 4 x 2
+// warps).  9 <= M <= 32: the swap-AB tcgen05 kernel (gemv_tc_kernel), whose
+// token columns grow for free.  Plans are fixed per shape (independent of
+// the device) so that workspace sizes are too.
 struct GemvPlan {
     bool tc;           // tcgen05 swap-AB kernel
     // register kernel
     int tg;            // token groups of 8
-    int ctas_x;        // CTAs along the rows (4 row blocks each)
+    int wn;            // row blocks per CTA (4, 2 or 1; 8 / wn warps along K)
+    int ctas_x;        // CTAs along the rows
     int nkseg;         // CTAs along K
+    int trig;          // early launch of the next kernel
     // tcgen05 kernel
     int bn, grid, ngroups, nkb;
     size_t part_bytes;
     int counters;
 };
 
-constexpr int kGemvWN = 4, kGemvWK = 2, kGemvUnrollDecode = 4, kGemvMinBlocks = 4;
+constexpr int kGemvUnrollDecode = 4, kGemvMinBlocks = 4;
 constexpr int kGemvGrid = 148;
 constexpr int kGemvMaxM = 32;
 
@@ -230,13 +239,19 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
     if (!g.tc) {
         g.tg = 1;
         const int64_t blocks = (N + 15) / 16;
-        g.ctas_x = (int)((blocks + kGemvWN - 1) / kGemvWN);
+        const int64_t slots = (int64_t)kGemvGrid * kGemvMinBlocks;
+        int wn = 4;
+        while (wn > 1 && (blocks + wn - 1) / wn * 2 < slots) wn /= 2;
+        g.wn = wn;
+        const int wk = 8 / wn;
+        g.ctas_x = (int)((blocks + wn - 1) / wn);
         const int64_t nchunks = (K + 63) / 64;
         int s = 1;
-        while (s < 16 && (int64_t)g.ctas_x * (s + 1) * 10 <= (int64_t)kGemvGrid * kGemvMinBlocks * 7 &&
-               nchunks / (kGemvWK * (s + 1)) >= 8)
+        while ((int64_t)g.ctas_x * 2 < slots && s < 16 && (int64_t)g.ctas_x * (s + 1) * 10 <= slots * 7 &&
+               nchunks / (wk * (s + 1)) >= 8)
             ++s;
         g.nkseg = s;
+        g.trig = (int64_t)g.ctas_x * s * 4 >= slots * 3 ? 1 : 0;
         g.part_bytes = s > 1 ? align_up((size_t)s * blocks * g.tg * 32 * 16, 256) : 0;
         g.counters = s > 1 ? g.ctas_x : 0;
     } else {
@@ -307,7 +322,12 @@ int launch_gemv_reg(const GemvShape& a, const GemvEpiDense& e, const GemvPlan& g
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     pdl_config(cfg, at, after_quant);
-    return cuda_status(cudaLaunchKernelEx(&cfg, gemv_dense_kernel<kGemvWN, kGemvWK, TG, U, kGemvMinBlocks>, a, e));
+    GemvShape args = a;
+    args.trig = g.trig;
+    auto kern = g.wn == 4 ? gemv_dense_kernel<4, 2, TG, U, kGemvMinBlocks>
+              : g.wn == 2 ? gemv_dense_kernel<2, 4, TG, U, kGemvMinBlocks>
+                          : gemv_dense_kernel<1, 8, TG, U, kGemvMinBlocks>;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, args, e));
 }
 
 // gate_up GEMV of the dense MLP block, gated epilogue (same plan as the dense GEMV).
@@ -322,6 +342,7 @@ int launch_gemv_gated(const int8_t* qx, const float* sx, const int8_t* qw, const
     a.nchunks = (int)((K + 63) / 64);
     a.part = reinterpret_cast<int32_t*>(scratch);
     a.counters = gemv_counters(g, scratch);
+    a.trig = g.trig;
     GemvEpiGated e;
     e.sx = sx;
     e.sw = sw;
@@ -334,8 +355,10 @@ int launch_gemv_gated(const int8_t* qx, const float* sx, const int8_t* qw, const
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     pdl_config(cfg, at, after_quant);
-    return cuda_status(
-        cudaLaunchKernelEx(&cfg, gemv_gated_kernel<kGemvWN, kGemvWK, 1, kGemvUnrollDecode, kGemvMinBlocks>, a, e));
+    auto kern = g.wn == 4 ? gemv_gated_kernel<4, 2, 1, kGemvUnrollDecode, kGemvMinBlocks>
+              : g.wn == 2 ? gemv_gated_kernel<2, 4, 1, kGemvUnrollDecode, kGemvMinBlocks>
+                          : gemv_gated_kernel<1, 8, 1, kGemvUnrollDecode, kGemvMinBlocks>;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, a, e));
 }
 
 // Runs the GEMV; `scratch` holds the partials and the counters (zero on entry).
@@ -664,7 +687,8 @@ int w8a8_linear(const uint16_t* x, const int8_t* qw, const float* sw, uint16_t* 
     int* ctr = gemv ? gemv_counters(g, scratch) : nullptr;
     if (K / 8 > (int64_t)8 * 256 * kQuantMaxVec) return W8A8_ERR_UNSUPPORTED;
     cudaError_t e =
-        launch_quant_rows<uint16_t>(x, M, K, K, qx, K, sx, st, current_sms(), ctr, ctr ? gemv_counter_count(g) : 0);
+        launch_quant_rows<uint16_t>(x, M, K, K, qx, K, sx, st, current_sms(), ctr, ctr ? gemv_counter_count(g) : 0,
+                                    true);
     if (e != cudaSuccess) return W8A8_ERR_CUDA;
     if (gemv) return run_gemv(qx, sx, qw, sw, y, M, N, K, false, g, scratch, true, st);
     return run_tc(qx, sx, qw, sw, y, M, N, K, kEpiBf16, st);
@@ -983,8 +1007,8 @@ int w8a8_mlp_forward(const uint16_t* x, const int8_t* w13, const float* s13, con
     int* ctr2 = gemv ? gemv_counters(g2, w.scratch2) : nullptr;
     int rc;
     // a1 (it also clears the gate_up GEMV's counters)
-    if (launch_quant_rows<uint16_t>(x, M, H, H, w.qx, H, w.sx, st, current_sms(), ctr1, ctr1 ? g1.counters : 0) !=
-        cudaSuccess)
+    if (launch_quant_rows<uint16_t>(x, M, H, H, w.qx, H, w.sx, st, current_sms(), ctr1, ctr1 ? g1.counters : 0,
+                                    true) != cudaSuccess)
         return W8A8_ERR_CUDA;
     // gate_up GEMM with SiLU(gate) * up -> fp32 a [M, I]
     if (gemv) {
@@ -1002,8 +1026,8 @@ int w8a8_mlp_forward(const uint16_t* x, const int8_t* w13, const float* s13, con
     }
     if (rc != W8A8_OK) return rc;
     // a9 (it also clears the down GEMV's counters)
-    if (launch_quant_rows<float>(w.a, M, I, I, w.qa, I, w.sa, st, current_sms(), ctr2, ctr2 ? g2.counters : 0) !=
-        cudaSuccess)
+    if (launch_quant_rows<float>(w.a, M, I, I, w.qa, I, w.sa, st, current_sms(), ctr2, ctr2 ? g2.counters : 0,
+                                 true) != cudaSuccess)
         return W8A8_ERR_CUDA;
     // down GEMM with the dense dequant
     rc = gemv ? run_gemv(w.qa, w.sa, w2, s2, y, M, H, I, false, g2, w.scratch2, true, st)
