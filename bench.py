@@ -4,10 +4,12 @@ Default workload (one "step"): one decode step of the two dense W8A8 linears
 of a Qwen3.6-27B-class MLP at M = 8 tokens -- gate_up (K=5120 -> N=34816) and
 down (K=17408 -> N=5120) -- each a per-token activation quant followed by the
 weight-streaming GEMV with the dequant epilogue.  The headline metric is the
-weight bytes streamed per second.  The same JSON line carries, under "extra",
-the prefill GEMM TOPS (M = 512 / 4096), the routed-MoE layer tokens/s
-(T = 1 / 8 / 512 / 4096) and the FWHT128-domain linear, each with its
-roofline fraction.
+weight bytes streamed per second.  Two independent weight sets alternate
+from step to step, so that no step finds its weights in L2.  The same JSON
+line carries, last, a compact "workloads" object: the prefill GEMM TOPS
+(M = 512 / 4096), the routed-MoE layer tokens/s (T = 1 / 8 / 512 / 4096), the
+FWHT128-domain, head, trunk, shared-expert and MLP-block workloads, each with
+its time and roofline fractions against the measured and the nominal peaks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--quick]   (headline only, no extra workloads)
@@ -33,6 +35,12 @@ sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "W8A8 int8 TOPS (prefill), weight GB/s (decode), MoE layer tokens/s vs roofline"
+# Nominal peaks of the part (HGX B200 datasheet, dense): HBM3e ~8 TB/s; int8
+# tensor ~4.5 POPS.  Every fraction is also reported against these.
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_INT8_TOPS = 4500.0
+DECODE_M = 8
+WEIGHT_SETS = 2       # ceil(2 * 126 MB / 267 MB) + 1: no step finds its weights in L2
 
 
 # --------------------------------------------------------------------------- peaks / clocks
@@ -236,27 +244,78 @@ def linear_bytes(M, N, K):
     return N * K + 4 * N + 2 * M * K + 2 * M * N
 
 
+def headline_config(world):
+    """The workload both arms measure (the reference arm on the host's cores)."""
+    return {"workload": "decode-shaped dense W8A8 linears, M=8 tokens: gate_up K=5120->N=34816 then "
+                        "down K=17408->N=5120 (per-token act quant + weight-streaming GEMV + dequant)",
+            "arithmetic": "int8 x int8 -> int32, fp32 scales, bf16 in/out",
+            "tokens": DECODE_M, "weight_bytes_per_step": 267546624, "algorithmic_bytes_per_step": 268546048,
+            "l2": f"{WEIGHT_SETS} weight sets of 267 MB alternate step by step (L2 126 MB): no step finds "
+                  "its weights in L2",
+            "parallelism": f"replicas x{world}"}
+
+
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def sig(v, n=4):
+    """v rounded to n significant digits (compact JSON)."""
+    if v is None or not np.isfinite(v) or v == 0:
+        return v
+    return float(f"{v:.{n}g}")
+
+
+def cnum(v):
+    """Compact number for the workloads record: integers from 100 up, else 3 significant digits."""
+    if v is None or not np.isfinite(v):
+        return v
+    return int(round(v)) if abs(v) >= 100 else sig(v, 3)
+
+
 # --------------------------------------------------------------------------- reference arm (CPU oracle)
+def decode_weights_np(inputs, oracle, seed=0):
+    """The headline's first weight set, quantized by the oracle (same draws as the GPU arm's set 0)."""
+    rng = np.random.default_rng([seed, 7])
+    out = {}
+    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
+        w = inputs.weights(rng, (d["N"], d["K"]))
+        out[name] = oracle.quant_rows_f32(w)
+        del w
+    return out
+
+
 def run_reference(args, rank, world):
+    """The CPU oracle, as it stands, on the whole decode step (both linears, all
+    rows) at the host's thread count; rank 0 only."""
     if rank != 0:
         return None
     import oracle
     from moe_gemm_absmax_b200 import inputs
     oracle.build()
+    oracle.set_threads(host_threads())
     cores = oracle.get_threads()
-    M = 8
-    rng = np.random.default_rng([0, 7])
-    rows = {"gate_up": 1024, "down": 256}         # bounded sample of each weight matrix's rows
-    mats = {}
-    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
-        w = inputs.weights(rng, (rows[name], d["K"]))
-        mats[name] = oracle.quant_rows_f32(w)
-    xs = {n: inputs.dense_linear(1, M, d["K"], 16, with_weights=False)[0]
+    mats = decode_weights_np(inputs, oracle)
+    xs = {n: inputs.dense_linear(11, DECODE_M, d["K"], 16, with_weights=False)[0]
           for n, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN))}
     wbytes = sum(mats[n][0].size + 4 * mats[n][0].shape[0] for n in mats)
 
     def step():
-        for n in mats:
+        for n in ("gate_up", "down"):
             oracle.linear(xs[n], *mats[n])
     for _ in range(args.warmup):
         step()
@@ -265,37 +324,100 @@ def run_reference(args, rank, world):
         step()
     dt = (time.perf_counter() - t0) / args.steps
     value = wbytes / dt / 1e9
-    sample = (f"decode step at M=8 on the first {rows['gate_up']} of 34816 gate_up rows and "
-              f"{rows['down']} of 5120 down rows; GB/s of those weight bytes")
+    sample = (f"the whole decode step (all 34816 gate_up and 5120 down rows, M=8) per step, "
+              f"one weight set (caches play no part on the host); {cores} threads, {cpu_model()}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": {"workload": "decode-shaped dense W8A8 linears, M=8 (gate_up 5120->34816, "
-                                   "down 17408->5120), CPU oracle on a row sample",
-                       "arithmetic": "int8 x int8 -> int32, fp32 scales, bf16 out"},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "config": headline_config(world),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
 
 
-def cpu_baseline(budget_s=12.0):
-    """The oracle, as it stands, on a bounded sample of the decode workload."""
+def _per_call(fn, min_s):
+    """Seconds per call of fn, timed over at least min_s after one untimed call."""
+    fn()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            return dt / n
+
+
+def cpu_baseline(min_s=1.0):
+    """The oracle, as it stands, on a bounded sample of each of the five
+    workloads, at one thread and at every thread of this process's affinity
+    mask.  Rates (GB/s, TOPS, tokens/s) of the sampled work; the headline value
+    is the decode step's GB/s at all threads."""
     import oracle
     from moe_gemm_absmax_b200 import inputs
     oracle.build()
+    nthr = host_threads()
     rng = np.random.default_rng([0, 7])
-    w = inputs.weights(rng, (2048, inputs.GATE_UP["K"]))
+    cases = {}
+    # tiny: the whole config
+    xb, w = inputs.tiny_linear(0)
     qw, sw = oracle.quant_rows_f32(w)
-    xb = inputs.dense_linear(1, 8, inputs.GATE_UP["K"], 16, with_weights=False)[0]
-    oracle.linear(xb, qw, sw)
-    n, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < budget_s:
-        oracle.linear(xb, qw, sw)
-        n += 1
-    dt = (time.perf_counter() - t0) / n
-    return {"value": qw.size / dt / 1e9, "unit": "GB/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": f"gate_up decode linear at M=8 on 2048 of its 34816 weight rows, {n} calls in "
-                      f"{budget_s:.0f} s; GB/s of the sampled int8 weight bytes"}
+    cases["tiny"] = dict(unit="GOP/s", work=2.0 * 16 * 512 * 512 / 1e9, fn=lambda: oracle.linear(xb, qw, sw),
+                         sample="whole config: 16 x 512 -> 512")
+    # decode step: a row sample of both matrices at M = 8
+    rows = {"gate_up": 2048, "down": 512}
+    dm = {}
+    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
+        dm[name] = (inputs.dense_linear(11, DECODE_M, d["K"], 16, with_weights=False)[0],
+                    *oracle.quant_rows_f32(inputs.weights(rng, (rows[name], d["K"]))))
+    dbytes = sum(dm[n][1].size + 4 * dm[n][1].shape[0] for n in dm)
+    cases["decode"] = dict(unit="GB/s", work=dbytes / 1e9,
+                           fn=lambda: [oracle.linear(*dm[n]) for n in ("gate_up", "down")],
+                           sample="decode step at M=8 on 2048 of 34816 gate_up rows and 512 of 5120 down rows; "
+                                  "GB/s of those weight bytes")
+    # prefill: M = 512 tokens against a row sample of gate_up
+    xp = inputs.dense_linear(3, 512, inputs.GATE_UP["K"], 16, with_weights=False)[0]
+    qp, sp = oracle.quant_rows_f32(inputs.weights(rng, (64, inputs.GATE_UP["K"])))
+    cases["prefill"] = dict(unit="TOPS", work=2.0 * 512 * 64 * inputs.GATE_UP["K"] / 1e12,
+                            fn=lambda: oracle.linear(xp, qp, sp),
+                            sample="prefill gate_up at M=512 on 64 of its 34816 weight rows")
+    # MoE at T = 8: the routed experts' weights only (drawn for the experts the tokens touch)
+    E, H, I, k = inputs.MOE["E"], inputs.MOE["H"], inputs.MOE["I"], inputs.MOE["topk"]
+    xm, lm = inputs.moe_tokens(0, 8)
+    ids, _ = oracle.route(lm, k)
+    w13 = np.zeros((E, 2 * I, H), np.int8)
+    w2 = np.zeros((E, H, I), np.int8)
+    s13 = np.ones((E, 2 * I), np.float32)
+    s2 = np.ones((E, H), np.float32)
+    mrng = np.random.default_rng([0, 1])
+    for e in np.unique(ids):
+        w13[e], s13[e] = oracle.quant_rows_f32(inputs.weights(mrng, (2 * I, H)))
+        w2[e], s2[e] = oracle.quant_rows_f32(inputs.weights(mrng, (H, I)))
+    cases["moe"] = dict(unit="tokens/s", work=8.0, fn=lambda: oracle.moe_forward(xm, lm, w13, s13, w2, s2, k),
+                        sample=f"routed MoE layer at T=8 ({len(np.unique(ids))} touched experts), whole layer")
+    # Hadamard: M = 2048, the rotation and group quant of x plus the GEMM on a row sample
+    xh, wh = inputs.hadamard_linear(2048, 2048)
+    qwh, swh, _ = oracle.fwht128_quant(wh[:64])
+
+    def had():
+        qx, sx, _ = oracle.fwht128_quant(xh)
+        oracle.gemm_g128(qx, sx, qwh, swh)
+    cases["hadamard"] = dict(unit="TOPS", work=2.0 * 2048 * 64 * 2048 / 1e12, fn=had,
+                             sample="FWHT128 linear at M=2048: rotation + group quant of x, GEMM on 64 of "
+                                    "4096 weight rows")
+    out = {}
+    for name, c in cases.items():
+        rec = {"unit": c["unit"], "sample": c["sample"]}
+        for label, n in (("t1", 1), ("tall", nthr)):
+            oracle.set_threads(n)
+            dt = _per_call(c["fn"], min_s)
+            rec[label] = sig(c["work"] / dt)
+        out[name] = rec
+    oracle.set_threads(nthr)
+    dec = out["decode"]
+    return {"value": dec["tall"], "unit": "GB/s", "cores": nthr, "kind": "oracle",
+            "sample": dec["sample"] + f"; {nthr} threads (sched_getaffinity)",
+            "cpu_model": cpu_model(), "threads_one": 1, "threads_all": nthr, "configs": out}
 
 
 # --------------------------------------------------------------------------- our arm
@@ -305,8 +427,9 @@ def run_ours(args, rank, world, torch, dev):
     peaks = load_peaks()
     hbm = peaks["hbm_gbs"]
     int8_peak = 2.0 * peaks["bf16_tflops"]           # dense int8 = 2 x dense bf16 (nominal ratio)
-    M = 8
-    W = dense_weights(torch, w8a8, inputs, dev)
+    M = DECODE_M
+    sets = [dense_weights(torch, w8a8, inputs, dev, seed=s) for s in range(WEIGHT_SETS)]
+    W = sets[0]
     xs = {}
     for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
         xs[name] = bf16_dev(torch, inputs.dense_linear(11, M, d["K"], 16, with_weights=False)[0], dev)
@@ -315,20 +438,20 @@ def run_ours(args, rank, world, torch, dev):
                           dtype=torch.uint8, device=dev) for n in W}
     order = ("gate_up", "down")
 
-    def step():
+    def step(i):
+        Ws = sets[i % WEIGHT_SETS]
         for n in order:
-            w8a8.linear(xs[n], W[n][0], W[n][1], y=ys[n], ws=wss[n])
+            w8a8.linear(xs[n], Ws[n][0], Ws[n][1], y=ys[n], ws=wss[n])
 
     step_bytes = sum(linear_bytes(M, W[n][0].shape[0], W[n][0].shape[1]) for n in order)
     weight_bytes = sum(W[n][0].numel() + 4 * W[n][0].shape[0] for n in order)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
+    for i in range(max(args.warmup, 3)):
+        step(i)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     # nvidia-smi samples every 100 ms; the timed loop alone is a few ms, so the
-    # sampler runs across the whole GPU part of the benchmark (timed loop,
-    # kernel-alone timing, end-to-end and the extra workloads)
+    # sampler runs across the whole GPU part of the benchmark
     clk = ClockSampler(local_gpu_index(torch))
     clk.__enter__()
     if world > 1:
@@ -337,12 +460,12 @@ def run_ours(args, rank, world, torch, dev):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     # a device-side sleep ahead of the start event keeps the GPU busy while the
-    # host enqueues the K steps (~20 us of host time each), so no launch gap of
-    # the host falls inside the timed region; the region itself is the K steps
+    # host enqueues the K steps, so no launch gap of the host falls inside the
+    # timed region; the region itself is the K steps
     torch.cuda._sleep(int(min(2e8, 60e3 * args.steps + 2e6)))
     e0.record(st)
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        step(i)
     e1.record(st)
     torch.cuda.synchronize()
     if world > 1:
@@ -358,14 +481,15 @@ def run_ours(args, rank, world, torch, dev):
     kfn = lambda: w8a8.gemm_q(qx, sx, W["gate_up"][0], W["gate_up"][1], w8a8.PATH_GEMV, y=y_k)
     for _ in range(3):
         kfn()
-    k_ms, k_med = time_events(torch, kfn, 20, flush=flush)
+    k_ms, _ = time_events(torch, kfn, 20, flush=flush)
     k_bytes = N * K + 4 * N + M * K + 4 * M + 2 * M * N
     achieved = k_bytes / (k_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": recorded_traffic(), "algorithmic_bytes": k_bytes,
-                "kernel": "gemv_dense_kernel<4,2,1,4,4> (gate_up K=5120 -> N=34816, M=8)",
+                "kernel": "gemv_dense_kernel (gate_up K=5120 -> N=34816, M=8)",
                 "timing": "kernel alone, CUDA events per launch, L2 evicted by a read between launches",
-                "peak_source": peaks["source"] + " (burst copy)"}
+                "peak_source": peaks["source"] + " (burst copy)",
+                "nominal_peak": NOMINAL_HBM_GBS, "nominal_frac": achieved / NOMINAL_HBM_GBS}
 
     # ---- the down-proj GEMV alone, and the whole step replayed from a CUDA graph
     qxd, sxd = w8a8.quant_act(xs["down"])
@@ -376,63 +500,73 @@ def run_ours(args, rank, world, torch, dev):
         dfn()
     d_ms, _ = time_events(torch, dfn, 20, flush=flush)
     d_bytes = Nd * Kd + 4 * Nd + M * Kd + 4 * M + 2 * M * Nd
-    graph_ms = graph_events(torch, step, 20)
+    graph_ms = graph_events(torch, lambda: [step(i) for i in range(WEIGHT_SETS)], 20) / WEIGHT_SETS
 
     # ---- end to end through the C ABI with host buffers: pinned x in, y out, each step
     hx = {n: xs[n].cpu().pin_memory() for n in order}
     hy = {n: torch.empty(ys[n].shape, dtype=torch.bfloat16).pin_memory() for n in order}
     dx = {n: torch.empty_like(xs[n]) for n in order}
 
-    def e2e_step():
+    def e2e_step(i):
+        Ws = sets[i % WEIGHT_SETS]
         for n in order:
             dx[n].copy_(hx[n], non_blocking=True)
-            w8a8.linear(dx[n], W[n][0], W[n][1], y=ys[n], ws=wss[n])
+            w8a8.linear(dx[n], Ws[n][0], Ws[n][1], y=ys[n], ws=wss[n])
             hy[n].copy_(ys[n], non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
+    for i in range(3):
+        e2e_step(i)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(st)
-    for _ in range(args.steps):
-        e2e_step()
+    for i in range(args.steps):
+        e2e_step(i)
     b.record(st)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / args.steps
     h2d = sum(hx[n].numel() * 2 for n in order)
     d2h = sum(hy[n].numel() * 2 for n in order)
 
-    extra = {} if args.quick else run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush)
+    def rec(ms_, val, peak, nominal, extra_ms=None):
+        r = [cnum(ms_ * 1e3), cnum(val), cnum(val / peak), cnum(val / nominal)]
+        return r if extra_ms is None else r + [cnum(extra_ms * 1e3)]
+
+    wl = {"dec_step_graph": rec(graph_ms, weight_bytes / (graph_ms * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS),
+          "dec_gu_gemv": rec(k_ms, achieved, hbm, NOMINAL_HBM_GBS),
+          "dec_dn_gemv": rec(d_ms, d_bytes / (d_ms * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS)}
+    if not args.quick:
+        del sets
+        wl.update(run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush, rec))
     clk.__exit__(None, None, None)
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": {"workload": "decode-shaped dense W8A8 linears, M=8 tokens: gate_up K=5120->N=34816 then "
-                                   "down K=17408->N=5120 (per-token act quant + weight-streaming GEMV + dequant)",
-                       "arithmetic": "int8 x int8 -> int32, fp32 scales, bf16 in/out",
-                       "tokens": M, "weight_bytes_per_step": weight_bytes, "algorithmic_bytes_per_step": step_bytes,
-                       "l2": "inputs larger than L2: 267 MB of weights streamed per step vs 126 MB L2",
-                       "parallelism": f"replicas x{world}"},
+            "config": headline_config(world),
+            "gpu_name": torch.cuda.get_device_name(dev),
+            "step_frac": {"measured": value / world / hbm, "nominal": value / world / NOMINAL_HBM_GBS,
+                          "bytes": "int8 weights + fp32 scales per step"},
             "roofline": roofline, "clocks": dict(clk.summary(), window="whole GPU part of the run"),
             "e2e": {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 4 * args.steps, "extra": extra}
-    line["decode_detail"] = {
-        "down_gemv_alone": {"kernel": "gemv_dense_kernel<4,2,1,4,4> (down K=17408 -> N=5120, M=8)", "ms": d_ms,
-                            "gbs": d_bytes / (d_ms * 1e-3) / 1e9, "frac": d_bytes / (d_ms * 1e-3) / 1e9 / hbm,
-                            "algorithmic_bytes": d_bytes},
-        "gate_up_gemv_alone_ms": k_ms,
-        "step_graph_replay": {"ms_per_step": graph_ms, "value": weight_bytes / (graph_ms * 1e-3) / 1e9,
-                              "unit": "GB/s", "note": "the same step captured once in a CUDA graph, replayed"}}
+            "gpu_launches": 4 * args.steps,
+            "peaks": {"hbm_gbs": hbm, "int8_tops": int8_peak, "source": peaks["source"],
+                      "nominal_hbm_gbs": NOMINAL_HBM_GBS, "nominal_int8_tops": NOMINAL_INT8_TOPS},
+            "workloads_fields": ["us", "value", "frac_measured", "frac_nominal",
+                                 "pf: us of a1 + GEMM; moe1/moe8: us of a CUDA-graph replay; had2048: us of "
+                                 "fwht128_quant + GEMM (the first four: the GEMM alone)"],
+            "workloads_units": {"dec": "GB/s", "pf": "TOPS", "mlp8": "GB/s", "mlp4096": "TOPS", "aq": "GB/s",
+                                "moe/moeg": "tokens/s (fractions: HBM bytes of the touched experts)",
+                                "had1/head/trunk1/shx1/shx8": "GB/s", "had2048/trunk2048/shx512/shx4096": "TOPS"},
+            "workloads": wl}
     return line
 
 
-def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
+def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush, rec):
     out = {}
-    # ---- prefill GEMMs (tcgen05), full linear incl. activation quant
+    # ---- prefill GEMMs (tcgen05), and the full linear incl. activation quant
     for M in (512, 4096):
-        for n in ("gate_up", "down"):
+        for n, tag in (("gate_up", "gu"), ("down", "dn")):
             N, K = W[n][0].shape
             x = bf16_dev(torch, inputs.dense_linear(3, M, K, 16, with_weights=False)[0], dev)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -446,12 +580,7 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
             t_lin, _ = time_events(torch, fn_lin, 10, flush=flush)
             t_gemm, _ = time_events(torch, fn_gemm, 10, flush=flush)
             ops = 2.0 * M * N * K
-            out[f"prefill_{n}_M{M}"] = {
-                "linear_ms": t_lin, "linear_tops": ops / (t_lin * 1e-3) / 1e12,
-                "gemm_ms": t_gemm, "gemm_tops": ops / (t_gemm * 1e-3) / 1e12,
-                "roofline": {"bound": "tensor", "achieved": ops / (t_gemm * 1e-3) / 1e12, "peak": int8_peak,
-                             "unit": "TOPS", "frac": ops / (t_gemm * 1e-3) / 1e12 / int8_peak,
-                             "peak_source": "2 x measured bf16 burst (dense int8 : bf16 = 2 : 1)"}}
+            out[f"pf_{tag}{M}"] = rec(t_gemm, ops / (t_gemm * 1e-3) / 1e12, int8_peak, NOMINAL_INT8_TOPS, t_lin)
             del x, y, ws, qx, sx
     # ---- dense gated MLP block: the same two matrices as gate_up (w13) and down (w2)
     q13, s13 = W["gate_up"]
@@ -468,15 +597,10 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         t, _ = time_events(torch, fn, 10, flush=flush)
         wbytes = q13.numel() + q2.numel() + 4 * (q13.shape[0] + H)
         ops = 2.0 * M * (2 * I) * H + 2.0 * M * H * I
-        rec = {"ms": t, "weight_gbs": wbytes / (t * 1e-3) / 1e9, "tops": ops / (t * 1e-3) / 1e12}
         if M == 8:
-            tg = graph_events(torch, fn, 10, flush=flush)
-            rec["graph_replay_ms"] = tg
-            rec["roofline"] = {"bound": "hbm", "frac": rec["weight_gbs"] / hbm, "peak": hbm, "unit": "GB/s",
-                               "bytes": wbytes}
+            out["mlp8"] = rec(t, wbytes / (t * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS)
         else:
-            rec["roofline"] = {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"}
-        out[f"mlp_M{M}"] = rec
+            out["mlp4096"] = rec(t, ops / (t * 1e-3) / 1e12, int8_peak, NOMINAL_INT8_TOPS)
         del x, y, ws
     # ---- per-token activation quant alone (a1) at the prefill shape
     for K in (5120, 17408):
@@ -486,9 +610,7 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
             qfn()
         tq, _ = time_events(torch, qfn, 10, flush=flush)
         qb = 4096 * K * 3 + 4096 * 4
-        out[f"act_quant_M4096_K{K}"] = {"ms": tq, "gbs": qb / (tq * 1e-3) / 1e9,
-                                        "roofline": {"bound": "hbm", "frac": qb / (tq * 1e-3) / 1e9 / hbm,
-                                                     "bytes": qb, "peak": hbm, "unit": "GB/s"}}
+        out[f"aq4096x{K}"] = rec(tq, qb / (tq * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS)
         del xq_in
     # ---- routed MoE layer
     w13, w2 = inputs.moe_weights(0)
@@ -499,6 +621,13 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
     g2 = w8a8.fwht128_quant(bf16_dev(torch, inputs.to_bf16_bits(w2).reshape(-1, w2.shape[2]), dev))
     del w13, w2
     E, I2, H = q13.shape
+
+    def moe_rec(t, T, touched, per_expert, tg=None):
+        byts = touched * per_expert + 2 * T * H * 2 + 2 * T * E
+        gbs = byts / (t * 1e-3) / 1e9
+        r = [cnum(t * 1e3), cnum(T / (t * 1e-3)), cnum(gbs / hbm), cnum(gbs / NOMINAL_HBM_GBS)]
+        return r if tg is None else r + [cnum(tg * 1e3)]
+
     per_expert = q13[0].numel() + q2[0].numel() + 4 * (I2 + H)
     for T in (1, 8, 512, 4096):
         xb, lb = inputs.moe_tokens(0, T)
@@ -509,15 +638,10 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         for _ in range(3):
             fn()
         t, _ = time_events(torch, fn, 10, flush=flush)
-        tg = graph_events(torch, fn, 10, flush=flush)
         _, dbg = w8a8.moe_forward(x, lg, q13, s13, q2, s2, 8, debug=True)
         touched = int((dbg["counts"] > 0).sum().item())
-        byts = touched * per_expert + 2 * T * H * 2 + 2 * T * E
-        out[f"moe_T{T}"] = {"ms": t, "tokens_per_s": T / (t * 1e-3), "touched_experts": touched,
-                            "graph_replay_ms": tg, "graph_replay_tokens_per_s": T / (tg * 1e-3),
-                            "roofline": {"bound": "hbm", "achieved": byts / (t * 1e-3) / 1e9, "peak": hbm,
-                                         "unit": "GB/s", "frac": byts / (t * 1e-3) / 1e9 / hbm,
-                                         "bytes": byts}}
+        tg = graph_events(torch, fn, 10, flush=flush) if T <= 8 else None
+        out[f"moe{T}"] = moe_rec(t, T, touched, per_expert, tg)
         del x, lg, y, ws
     del q13, q2
     # ---- routed MoE layer on the FWHT128 grid
@@ -533,15 +657,9 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         for _ in range(3):
             fn()
         t, _ = time_events(torch, fn, 10, flush=flush)
-        tg = graph_events(torch, fn, 10, flush=flush)
         _, dbg = w8a8.moe_g128_forward(x, lg, gq13, gs13, gq2, gs2, 8, debug=True)
         touched = int((dbg["counts"] > 0).sum().item())
-        byts = touched * per_expert + 2 * T * H * 2 + 2 * T * E
-        out[f"moe_g128_T{T}"] = {"ms": t, "tokens_per_s": T / (t * 1e-3), "touched_experts": touched,
-                                 "graph_replay_ms": tg, "graph_replay_tokens_per_s": T / (tg * 1e-3),
-                                 "roofline": {"bound": "hbm", "achieved": byts / (t * 1e-3) / 1e9, "peak": hbm,
-                                              "unit": "GB/s", "frac": byts / (t * 1e-3) / 1e9 / hbm,
-                                              "bytes": byts}}
+        out[f"moeg{T}"] = moe_rec(t, T, touched, per_expert)
         del x, lg, y, ws
     del g13, g2, gq13, gs13, gq2, gs2
     # ---- FWHT128-domain linear
@@ -550,7 +668,6 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
     for M in (1, 2048):
         xb, _ = inputs.hadamard_linear(M, M)
         x = bf16_dev(torch, xb, dev)
-        qx, sx = w8a8.fwht128_quant(x)
         y = torch.empty((M, qw.shape[0]), dtype=torch.bfloat16, device=dev)
 
         def fn():
@@ -562,12 +679,15 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         N, K = qw.shape
         ops = 2.0 * M * N * K
         byts = N * K + 2 * N * (K // 128) + 2 * M * K + 2 * M * N
-        rec = {"ms": t, "tops": ops / (t * 1e-3) / 1e12, "gbs": byts / (t * 1e-3) / 1e9}
         if M == 1:
-            rec["roofline"] = {"bound": "hbm", "frac": rec["gbs"] / hbm, "peak": hbm, "unit": "GB/s"}
+            out["had1"] = rec(t, byts / (t * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS)
         else:
-            rec["roofline"] = {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"}
-        out[f"hadamard_M{M}"] = rec
+            q, s = w8a8.fwht128_quant(x)
+            gfn = lambda: w8a8.linear_g128(q, s, qw, sw, y=y)
+            for _ in range(3):
+                gfn()
+            tg, _ = time_events(torch, gfn, 10, flush=flush)
+            out["had2048"] = rec(tg, ops / (tg * 1e-3) / 1e12, int8_peak, NOMINAL_INT8_TOPS, t)
     # ---- head-shaped group-128 GEMM on the unrotated grid (N = 131072 rows, K = 2048)
     del qw, sw
     HN, HK = HEAD["N"], HEAD["K"]
@@ -586,9 +706,7 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
             fn()
         t, _ = time_events(torch, fn, 10, flush=flush)
         byts = HN * HK + 2 * HN * (HK // 128) + 2 * M * HK + 2 * M * HN
-        gbs = byts / (t * 1e-3) / 1e9
-        out[f"head_group128_M{M}"] = {"ms": t, "gbs": gbs, "roofline": {"bound": "hbm", "frac": gbs / hbm, "peak": hbm,
-                                                                         "unit": "GB/s", "bytes": byts}}
+        out[f"head{M}"] = rec(t, byts / (t * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS)
     del qw, sw
     # ---- trunk linear in the two-level format, on the Hadamard config's shapes (N = 4096, K = 2048)
     d = inputs.HADAMARD
@@ -608,10 +726,8 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         N, K = tq.shape
         ops = 2.0 * M * N * K
         byts = N * K + N * (K // 256) + 2 * N + 2 * M * K + 2 * M * N
-        rec = {"ms": t, "tops": ops / (t * 1e-3) / 1e12, "gbs": byts / (t * 1e-3) / 1e9}
-        rec["roofline"] = ({"bound": "hbm", "frac": rec["gbs"] / hbm, "peak": hbm, "unit": "GB/s"} if M == 1 else
-                           {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"})
-        out[f"trunk_M{M}"] = rec
+        out[f"trunk{M}"] = (rec(t, byts / (t * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS) if M == 1 else
+                            rec(t, ops / (t * 1e-3) / 1e12, int8_peak, NOMINAL_INT8_TOPS))
     del tq, tu8, ts2
     # ---- shared expert (gate_up in the trunk format, down on the group-128 grid), H = 2048, I = 512
     H, I = inputs.MOE["H"], inputs.MOE["I"]
@@ -632,11 +748,8 @@ def run_extra(torch, w8a8, inputs, dev, W, hbm, int8_peak, flush):
         t, _ = time_events(torch, fn, 10, flush=flush)
         ops = 2.0 * M * 3 * H * I
         byts = wbytes + 2 * M * H * 2
-        rec = {"ms": t, "tokens_per_s": M / (t * 1e-3), "tops": ops / (t * 1e-3) / 1e12,
-               "gbs": byts / (t * 1e-3) / 1e9}
-        rec["roofline"] = ({"bound": "hbm", "frac": rec["gbs"] / hbm, "peak": hbm, "unit": "GB/s"} if M <= 8 else
-                           {"bound": "tensor", "frac": rec["tops"] / int8_peak, "peak": int8_peak, "unit": "TOPS"})
-        out[f"shared_expert_M{M}"] = rec
+        out[f"shx{M}"] = (rec(t, byts / (t * 1e-3) / 1e9, hbm, NOMINAL_HBM_GBS) if M <= 8 else
+                          rec(t, ops / (t * 1e-3) / 1e12, int8_peak, NOMINAL_INT8_TOPS))
         del x, y, ws
     return out
 
@@ -782,6 +895,7 @@ def main():
     if rank == 0:
         if world == 1:
             line["cpu_baseline"] = cpu_baseline()
+        line["workloads"] = line.pop("workloads")   # the compact record goes last
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()
