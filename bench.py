@@ -357,24 +357,22 @@ def cpu_baseline(min_s=1.0):
     from moe_gemm_absmax_b200 import inputs
     oracle.build()
     nthr = host_threads()
-    rng = np.random.default_rng([0, 7])
+    rng = np.random.default_rng([0, 8])
     cases = {}
     # tiny: the whole config
     xb, w = inputs.tiny_linear(0)
     qw, sw = oracle.quant_rows_f32(w)
     cases["tiny"] = dict(unit="GOP/s", work=2.0 * 16 * 512 * 512 / 1e9, fn=lambda: oracle.linear(xb, qw, sw),
                          sample="whole config: 16 x 512 -> 512")
-    # decode step: a row sample of both matrices at M = 8
-    rows = {"gate_up": 2048, "down": 512}
-    dm = {}
-    for name, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN)):
-        dm[name] = (inputs.dense_linear(11, DECODE_M, d["K"], 16, with_weights=False)[0],
-                    *oracle.quant_rows_f32(inputs.weights(rng, (rows[name], d["K"]))))
+    # decode step: the whole step (both matrices, every row) at M = 8
+    mats = decode_weights_np(inputs, oracle)
+    dm = {n: (inputs.dense_linear(11, DECODE_M, d["K"], 16, with_weights=False)[0], *mats[n])
+          for n, d in (("gate_up", inputs.GATE_UP), ("down", inputs.DOWN))}
     dbytes = sum(dm[n][1].size + 4 * dm[n][1].shape[0] for n in dm)
     cases["decode"] = dict(unit="GB/s", work=dbytes / 1e9,
                            fn=lambda: [oracle.linear(*dm[n]) for n in ("gate_up", "down")],
-                           sample="decode step at M=8 on 2048 of 34816 gate_up rows and 512 of 5120 down rows; "
-                                  "GB/s of those weight bytes")
+                           sample="the whole decode step at M=8 (all 34816 gate_up and 5120 down rows), one "
+                                  "weight set; GB/s of its int8 weights and fp32 scales")
     # prefill: M = 512 tokens against a row sample of gate_up
     xp = inputs.dense_linear(3, 512, inputs.GATE_UP["K"], 16, with_weights=False)[0]
     qp, sp = oracle.quant_rows_f32(inputs.weights(rng, (64, inputs.GATE_UP["K"])))
