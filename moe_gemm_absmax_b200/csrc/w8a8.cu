@@ -166,6 +166,45 @@ int pick_tc2_bn(int64_t M, int64_t N, int clusters) {
     return cost(160) < cost(256) ? 160 : 256;
 }
 
+// Group-128 GEMM on pair tiles (256 x 128).
+int launch_tc2_g128(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
+    using SM = Tc2gSmem;
+    auto kern = gemm_i8_tc2_g128_kernel;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED;
+    static int max_clusters[kMaxDevices] = {0};
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kTc2gThreads, 1, 1);
+    cfg.dynamicSmemBytes = SM::kBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (max_clusters[dev] == 0) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+        cfg.gridDim = dim3((unsigned)(2 * (device_sms(dev) / 2)), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_sms(dev) / 2;
+        max_clusters[dev] = n;
+    }
+    CUtensorMap ta, tb;
+    if (!make_tmap_i8(&ta, A, (uint64_t)p.M, (uint64_t)p.K, 128)) return W8A8_ERR_CUDA;
+    if (!make_tmap_i8(&tb, B, (uint64_t)p.N, (uint64_t)p.K, kTc2gBN / 2)) return W8A8_ERR_CUDA;
+    p.num_m_tiles = (p.M + kTc2BM - 1) / kTc2BM;
+    p.num_n_tiles = (p.N + kTc2gBN - 1) / kTc2gBN;
+    p.num_k_blocks = (p.K + kTcBK - 1) / kTcBK;
+    const int tiles = p.num_m_tiles * p.num_n_tiles;
+    const int clusters = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, p));
+}
+
 template <int EPI>
 int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
     return pick_tc2_bn(p.M, p.N, current_sms() / 2) == 160 ? launch_tc2_bn<EPI, 160>(A, B, p, st)
@@ -1230,6 +1269,7 @@ int linear_group_scaled(const int8_t* qx, const uint16_t* sx, const int8_t* qw, 
     p.gsw_row = sw_row;
     p.gpost = post;
     p.out = y;
+    if (M >= kTc2MinM) return launch_tc2_g128(qx, qw, p, st);
     return launch_tc<128, 6, kEpiG128, 4, 8>(qx, qw, p, st);
 }
 

@@ -35,7 +35,7 @@ def test_fwht128_quant_weights_and_zero_blocks(orc):
     assert np.array_equal(from_dev_bf16(s), so)
 
 
-@pytest.mark.parametrize("M", [1, 5, 8, 2048, 200])
+@pytest.mark.parametrize("M", [1, 5, 8, 2048, 200, 300, 777])
 def test_linear_g128(orc, M):
     xb, wb = inputs.hadamard_linear(M + 11, M)
     qx, sx = _fwht_gpu(xb)
@@ -43,7 +43,7 @@ def test_linear_g128(orc, M):
     y = from_dev_bf16(w8a8.linear_g128(qx, sx, qw, sw))
     qxo, sxo, _ = orc.fwht128_quant(xb)
     qwo, swo, _ = orc.fwht128_quant(wb)
-    rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 48),
+    rows = np.arange(M) if M <= 2048 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 48),
                                                                   [0, 127, 128, M - 1]]))
     yo, y32 = orc.gemm_g128(qxo[rows], sxo[rows], qwo, swo)
     exact = assert_bf16_close(y[rows], y32, what=f"g128 M={M}")
@@ -63,7 +63,8 @@ def test_group128_quant_bit_exact(orc, M):
     assert np.array_equal(from_dev_bf16(s), so)
 
 
-@pytest.mark.parametrize("M,N", [(1, 4096), (4, 4096), (8, 1040), (9, 4096), (200, 1040), (2048, 4096)])
+@pytest.mark.parametrize("M,N", [(1, 4096), (4, 4096), (8, 1040), (9, 4096), (200, 1040), (2048, 4096),
+                                 (520, 1040), (256, 136)])
 def test_linear_group128(orc, M, N):
     xb, wb = inputs.hadamard_linear(M + 29, M, N=N)
     qx, sx = w8a8.group128_quant(to_dev_bf16(xb))
@@ -72,7 +73,7 @@ def test_linear_group128(orc, M, N):
     qxo, sxo = orc.group128_quant(xb)
     qwo, swo = orc.group128_quant(wb)
     assert np.array_equal(qw.cpu().numpy(), qwo) and np.array_equal(from_dev_bf16(sw), swo)
-    rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 48),
+    rows = np.arange(M) if M <= 2048 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 48),
                                                                   [0, 127, 128, M - 1]]))
     yo, y32 = orc.gemm_group128(qxo[rows], sxo[rows], qwo, swo)
     assert assert_bf16_close(y[rows], y32, what=f"group128 M={M}") == 1.0

@@ -1,7 +1,8 @@
 """GPU parity of the dense W8A8 path: int32 accumulators bit for bit
 (tcgen05 GEMM and weight-streaming GEMV), bf16 dequant outputs within one
 bf16 ulp of the oracle's fp32 value, at small ragged shapes and at the
-workload shapes (decode in full, prefill on sampled outputs)."""
+workload shapes (decode in full, prefill at M = 512 in full and at M = 4096
+on sampled outputs)."""
 import numpy as np
 import pytest
 import torch
@@ -94,6 +95,22 @@ def test_linear_prefill_full_size_sampled(orc, M, shape):
     y32 = (acc.astype(np.float32) * sx[ms]) * sw[ns]
     exact = assert_bf16_close(y[ms, ns], y32, what=f"prefill {shape} M={M}")
     assert exact == 1.0
+
+
+@pytest.mark.parametrize("shape", ["gate_up", "down"])
+def test_linear_prefill_m512_every_output(orc, shape):
+    """Every output of the prefill shape at M = 512 (2.6 M / 17.8 M values),
+    so that every tile of every wave of the persistent pair-tile scheduler is
+    compared, not a sample."""
+    d = inputs.GATE_UP if shape == "gate_up" else inputs.DOWN
+    K, N, M = d["K"], d["N"], 512
+    rng = np.random.default_rng(M + K + 1)
+    xb = inputs.dense_linear(300 + M, M, K, 16, with_weights=False)[0]
+    qw, sw = orc.quant_rows_f32(inputs.weights(rng, (N, K)))
+    y = from_dev_bf16(w8a8.linear(to_dev_bf16(xb), torch.from_numpy(qw).cuda(), torch.from_numpy(sw).cuda()))
+    yo, y32, _, _ = orc.linear(xb, qw, sw)
+    assert assert_bf16_close(y, y32, what=f"prefill {shape} M=512, every output") == 1.0
+    assert np.array_equal(y, yo)
 
 
 def test_linear_prefill_ragged_rows(orc):

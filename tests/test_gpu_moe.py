@@ -115,6 +115,14 @@ def test_moe_full_size(orc, full_experts, T):
     _compare(orc, xb, lb, gw, ow, 8, tokens)
 
 
+def test_moe_full_size_every_token_t512(orc, full_experts):
+    """Every token of the layer at T = 512 (4096 sorted rows over all 256
+    experts), not a sample: every token block of every expert."""
+    gw, ow = full_experts
+    xb, lb = inputs.moe_tokens(0, 512)
+    _compare(orc, xb, lb, gw, ow, 8, None)
+
+
 def test_moe_full_size_extreme_skew(orc, full_experts):
     """Every token's logits favour the same 8 experts: 512 rows each for those
     (many token blocks per expert on the swap-AB path), 0 for the other 248."""

@@ -38,14 +38,14 @@ def test_trunk_weight_quant_bit_exact(orc, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 512, 2048), (4, 1040, 512), (8, 4096, 2048), (9, 512, 2048),
-                                   (200, 1040, 512), (2048, 4096, 2048)])
+                                   (200, 1040, 512), (2048, 4096, 2048), (300, 1040, 512), (513, 264, 1024)])
 def test_linear_trunk(orc, M, N, K):
     xb, wb = inputs.hadamard_linear(M + N, M, K=K, N=N)
     (q, su8, s2), (qo, su8o, s2o) = _trunk_both(orc, wb)
     qx, sx = w8a8.fwht128_quant(to_dev_bf16(xb))
     y = from_dev_bf16(w8a8.linear_trunk(qx, sx, q, su8, s2))
     qxo, sxo, _ = orc.fwht128_quant(xb)
-    rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 40),
+    rows = np.arange(M) if M <= 2048 else np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 40),
                                                                   [0, 127, 128, M - 1]]))
     yo, y32 = orc.gemm_trunk(qxo[rows], sxo[rows], qo, su8o, s2o)
     assert assert_bf16_close(y[rows], y32, what=f"trunk M={M}") == 1.0
