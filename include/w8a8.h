@@ -156,6 +156,25 @@ typedef struct w8a8_moe_debug {
 } w8a8_moe_debug;
 
 W8A8_API size_t w8a8_moe_workspace_size(int64_t T, int E, int H, int I, int topk);
+
+/* How w8a8_moe_forward adds each token's k contributions (process-wide;
+ * no counterpart on the pages, which fix only the sum itself):
+ *   W8A8_MOE_COMBINE_AUTO (default)  in fp32 in slot order -- the definition's
+ *       order, bit-exact and deterministic -- while T * topk * H * 4 bytes of
+ *       contributions stay within 64 MiB; beyond that with fp32 atomics into
+ *       the token's row (order unspecified: within one bf16 ulp plus the
+ *       reordering bound of a k-term fp32 sum, not bit-exact, not
+ *       run-to-run deterministic), which saves an HBM round trip of the
+ *       [T * topk, H] contributions;
+ *   W8A8_MOE_COMBINE_EXACT           in slot order at every T.
+ * The mode also sizes the workspace (w8a8_moe_workspace_size): set it before
+ * sizing, and do not change it between sizing and the forward call (a call
+ * whose workspace is then too small returns W8A8_ERR_WORKSPACE).  Returns the
+ * previous mode, or W8A8_ERR_INVALID_ARG for an unknown one. */
+#define W8A8_MOE_COMBINE_AUTO 0
+#define W8A8_MOE_COMBINE_EXACT 1
+W8A8_API int w8a8_moe_set_combine(int mode);
+
 W8A8_API int w8a8_moe_forward(const uint16_t* x, const uint16_t* logits, const int8_t* w13, const float* s13,
                      const int8_t* w2, const float* s2, uint16_t* y, int64_t T, int E, int H, int I, int topk,
                      void* ws, size_t ws_bytes, const w8a8_moe_debug* dbg, void* stream);
@@ -246,6 +265,7 @@ W8A8_API int w8a8_trunk_weight_quant(const uint16_t* w, int64_t N, int64_t K, in
                                      void* stream);
 W8A8_API int w8a8_linear_trunk(const int8_t* qx, const uint16_t* sx, const int8_t* qw, const uint8_t* su8,
                                const uint16_t* s2, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
+
 
 /* ---------------------------------------------------------------------------
  * The shared expert -- [IQ8R] file table (Experts row: the shared expert is

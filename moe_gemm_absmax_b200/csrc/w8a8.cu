@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -496,7 +497,11 @@ struct MoeWs {
 // fits comfortably in L2; beyond that it accumulates with fp32 vector atomics
 // into [T, H] (order unspecified).
 constexpr size_t kMoeExactCombineBytes = (size_t)64 << 20;
-inline bool moe_exact_combine(int64_t R, int H) { return (size_t)R * H * 4 <= kMoeExactCombineBytes; }
+std::atomic<int> g_moe_combine{W8A8_MOE_COMBINE_AUTO};
+inline bool moe_exact_combine(int64_t R, int H) {
+    return g_moe_combine.load(std::memory_order_relaxed) == W8A8_MOE_COMBINE_EXACT ||
+           (size_t)R * H * 4 <= kMoeExactCombineBytes;
+}
 
 // Token blocks of the swap path: at most one partial block per touched expert.
 inline int64_t moe_max_blocks(int64_t R, int E, int bn) { return R / bn + (R < E ? R : E) + 1; }
@@ -847,6 +852,11 @@ int moe_debug_copies(const MoeWs& w, const w8a8_moe_debug* dbg, int64_t R, int E
 }  // namespace
 
 extern "C" {
+
+int w8a8_moe_set_combine(int mode) {
+    if (mode != W8A8_MOE_COMBINE_AUTO && mode != W8A8_MOE_COMBINE_EXACT) return W8A8_ERR_INVALID_ARG;
+    return g_moe_combine.exchange(mode);
+}
 
 size_t w8a8_moe_workspace_size(int64_t T, int E, int H, int I, int topk) {
     if (T <= 0 || E <= 0 || H <= 0 || I <= 0 || topk <= 0) return 0;

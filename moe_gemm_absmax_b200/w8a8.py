@@ -24,7 +24,7 @@ EXPORTS = (
     "w8a8_quant_act", "w8a8_quant_rows_f32", "w8a8_linear_workspace_size", "w8a8_linear",
     "w8a8_linear_noalloc_scratch_size", "w8a8_linear_noalloc",
     "w8a8_gemm_workspace_size", "w8a8_gemm_q", "w8a8_gemm_s32", "w8a8_moe_workspace_size",
-    "w8a8_moe_forward", "w8a8_moe_g128_workspace_size", "w8a8_moe_g128_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
+    "w8a8_moe_forward", "w8a8_moe_set_combine", "w8a8_moe_g128_workspace_size", "w8a8_moe_g128_forward", "w8a8_mlp_workspace_size", "w8a8_mlp_forward", "fwht128_quant", "w8a8_linear_g128",
     "group128_quant", "w8a8_linear_group128", "w8a8_trunk_weight_quant", "w8a8_linear_trunk",
     "w8a8_shared_expert_workspace_size", "w8a8_shared_expert_forward",
     "w8a8_exp_proj",
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         "w8a8_gemm_q": ([vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp], i32),
         "w8a8_gemm_s32": ([vp, vp, vp, i64, i64, i64, i32, vp, sz, vp], i32),
         "w8a8_moe_workspace_size": ([i64, i32, i32, i32, i32], sz),
+        "w8a8_moe_set_combine": ([i32], i32),
         "w8a8_moe_forward": ([vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, sz,
                               ctypes.POINTER(MoeDebug), vp], i32),
         "w8a8_moe_g128_workspace_size": ([i64, i32, i32, i32, i32], sz),
@@ -262,6 +263,17 @@ def gemm_s32(qx, qw, path: int = PATH_AUTO, acc=None, ws=None, stream=None) -> t
 
 def moe_workspace_size(T: int, E: int, H: int, I: int, topk: int) -> int:
     return int(lib().w8a8_moe_workspace_size(T, E, H, I, topk))
+
+
+MOE_COMBINE_AUTO, MOE_COMBINE_EXACT = 0, 1
+
+
+def moe_set_combine(mode: int) -> int:
+    """Combine mode of moe_forward (process-wide); returns the previous one."""
+    r = int(lib().w8a8_moe_set_combine(int(mode)))
+    if r < 0:
+        raise W8A8Error(r, "w8a8_moe_set_combine")
+    return r
 
 
 def moe_forward(x, logits, w13, s13, w2, s2, topk: int = 8, y=None, ws=None, debug: bool = False,

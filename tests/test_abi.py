@@ -47,6 +47,21 @@ def test_workspace_queries(L):
     assert L.w8a8_gemm_workspace_size(4096, 5120, 17408, w8a8.PATH_TCGEN05) == 0
 
 
+def test_moe_combine_mode(L):
+    auto = L.w8a8_moe_workspace_size(4096, 256, 2048, 512, 8)
+    assert w8a8.moe_set_combine(w8a8.MOE_COMBINE_EXACT) == w8a8.MOE_COMBINE_AUTO
+    try:
+        exact = L.w8a8_moe_workspace_size(4096, 256, 2048, 512, 8)
+        # the [T * topk, H] fp32 contributions instead of the [T, H] atomic buffer
+        assert exact - auto >= (4096 * 8 - 4096) * 2048 * 4
+        assert L.w8a8_moe_set_combine(7) == w8a8.ERR_INVALID_ARG
+    finally:
+        assert w8a8.moe_set_combine(w8a8.MOE_COMBINE_AUTO) == w8a8.MOE_COMBINE_EXACT
+    assert L.w8a8_moe_workspace_size(4096, 256, 2048, 512, 8) == auto
+    # small T: the slot-order combine either way
+    assert L.w8a8_moe_workspace_size(8, 256, 2048, 512, 8) > 8 * 8 * 2048 * 4
+
+
 def test_argument_checks_without_gpu(L):
     vp = ctypes.c_void_p
     fake = vp(0x10000)

@@ -31,7 +31,7 @@ def _quant_experts_orc(orc, w13, w2):
     return q13.reshape(w13.shape), s13.reshape(E, I2), q2.reshape(w2.shape), s2.reshape(E, H)
 
 
-def _compare(orc, xb, lb, gpu_w, orc_w, topk, tokens):
+def _compare(orc, xb, lb, gpu_w, orc_w, topk, tokens, exact=None):
     q13, s13, q2, s2 = gpu_w
     y, dbg = w8a8.moe_forward(to_dev_bf16(xb), to_dev_bf16(lb), q13, s13, q2, s2, topk, debug=True)
     y = from_dev_bf16(y)
@@ -48,7 +48,9 @@ def _compare(orc, xb, lb, gpu_w, orc_w, topk, tokens):
     assert np.array_equal(dbg["qa"].cpu().numpy()[t], ref["qa"])
     assert np.array_equal(dbg["sa"].cpu().numpy()[t].view(np.uint32), ref["sa"].view(np.uint32))
     H = xb.shape[1]
-    if xb.shape[0] * topk * H * 4 <= 64 << 20:
+    if exact is None:
+        exact = xb.shape[0] * topk * H * 4 <= 64 << 20
+    if exact:
         # slot-order combine: the oracle's fp32 steps exactly
         assert assert_bf16_close(y[t], ref["y32"], what="moe y") == 1.0
         assert np.array_equal(y[t], ref["y"])
@@ -113,6 +115,19 @@ def test_moe_full_size(orc, full_experts, T):
     rng = np.random.default_rng(T)
     tokens = None if T <= 8 else np.unique(np.concatenate([rng.integers(0, T, 24), [0, T - 1]]))
     _compare(orc, xb, lb, gw, ow, 8, tokens)
+
+
+def test_moe_full_size_exact_combine_t4096(orc, full_experts):
+    """With the slot-order combine forced at every T, the T = 4096 layer is
+    bit-exact with the oracle's bf16 on the sampled tokens."""
+    gw, ow = full_experts
+    xb, lb = inputs.moe_tokens(0, 4096)
+    tokens = np.unique(np.concatenate([np.random.default_rng(41).integers(0, 4096, 24), [0, 4095]]))
+    prev = w8a8.moe_set_combine(w8a8.MOE_COMBINE_EXACT)
+    try:
+        _compare(orc, xb, lb, gw, ow, 8, tokens, exact=True)
+    finally:
+        w8a8.moe_set_combine(prev)
 
 
 def test_moe_full_size_every_token_t512(orc, full_experts):
