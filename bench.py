@@ -500,31 +500,71 @@ def run_ours(args, rank, world, torch, dev):
     d_bytes = Nd * Kd + 4 * Nd + M * Kd + 4 * M + 2 * M * Nd
     graph_ms = graph_events(torch, lambda: [step(i) for i in range(WEIGHT_SETS)], 20) / WEIGHT_SETS
 
-    # ---- end to end through the C ABI with host buffers: pinned x in, y out, each step
-    hx = {n: xs[n].cpu().pin_memory() for n in order}
-    hy = {n: torch.empty(ys[n].shape, dtype=torch.bfloat16).pin_memory() for n in order}
-    dx = {n: torch.empty_like(xs[n]) for n in order}
-
-    def e2e_step(i):
-        Ws = sets[i % WEIGHT_SETS]
+    # ---- end to end through the C ABI with host buffers: every step's x comes
+    # from pinned host memory and its y goes back to it, the copies on a second
+    # stream one step ahead / behind the compute (a serving loop's pipeline),
+    # both inputs in one host-to-device copy and both outputs in one back
+    xbytes = {n: xs[n].numel() * 2 for n in order}
+    ybytes = {n: ys[n].numel() * 2 for n in order}
+    h2d = sum(xbytes.values())
+    d2h = sum(ybytes.values())
+    hx = [torch.empty(h2d, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    hy = [torch.empty(d2h, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    for slot in range(2):
+        o = 0
         for n in order:
-            dx[n].copy_(hx[n], non_blocking=True)
-            w8a8.linear(dx[n], Ws[n][0], Ws[n][1], y=ys[n], ws=wss[n])
-            hy[n].copy_(ys[n], non_blocking=True)
+            hx[slot][o:o + xbytes[n]].copy_(xs[n].view(torch.uint8).reshape(-1).cpu())
+            o += xbytes[n]
+    dxb = [torch.empty(h2d, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dyb = [torch.empty(d2h, dtype=torch.uint8, device=dev) for _ in range(2)]
 
-    for i in range(3):
-        e2e_step(i)
+    def view_bf16(buf, sizes, shapes):
+        out, o = {}, 0
+        for n in order:
+            out[n] = buf[o:o + sizes[n]].view(torch.bfloat16).view(shapes[n])
+            o += sizes[n]
+        return out
+    dx = [view_bf16(dxb[k], xbytes, {n: xs[n].shape for n in order}) for k in range(2)]
+    dy = [view_bf16(dyb[k], ybytes, {n: ys[n].shape for n in order}) for k in range(2)]
+    cs = torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_run(nsteps):
+        cs.wait_stream(st)   # the copies start inside the timed region
+        with torch.cuda.stream(cs):
+            dxb[0].copy_(hx[0], non_blocking=True)
+            ev_in[0].record(cs)
+        for i in range(nsteps):
+            k = i % 2
+            if i + 1 < nsteps:
+                with torch.cuda.stream(cs):   # next step's x, once step i - 1 is done with that slot
+                    dxb[1 - k].copy_(hx[1 - k], non_blocking=True)
+                    ev_in[1 - k].record(cs)
+            st.wait_event(ev_in[k])
+            if i >= 2:
+                st.wait_event(ev_out[k])      # step i - 2's y has left that slot
+            Ws = sets[i % WEIGHT_SETS]
+            for n in order:
+                w8a8.linear(dx[k][n], Ws[n][0], Ws[n][1], y=dy[k][n], ws=wss[n])
+            ev_done[k].record(st)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_done[k])
+                hy[k].copy_(dyb[k], non_blocking=True)
+                ev_out[k].record(cs)
+        st.wait_stream(cs)
+
+    e2e_run(3)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(min(2e8, 60e3 * args.steps + 2e6)))
     a.record(st)
-    for i in range(args.steps):
-        e2e_step(i)
+    e2e_run(args.steps)
     b.record(st)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / args.steps
-    h2d = sum(hx[n].numel() * 2 for n in order)
-    d2h = sum(hy[n].numel() * 2 for n in order)
 
     def rec(ms_, val, peak, nominal, extra_ms=None):
         r = [cnum(ms_ * 1e3), cnum(val), cnum(val / peak), cnum(val / nominal)]
@@ -546,7 +586,9 @@ def run_ours(args, rank, world, torch, dev):
                           "bytes": "int8 weights + fp32 scales per step"},
             "roofline": roofline, "clocks": dict(clk.summary(), window="whole GPU part of the run"),
             "e2e": {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "how": "pinned host x in and y out every step (one copy each way), on a copy stream "
+                           "pipelined one step ahead of / behind the compute"},
             "gpu_launches": 4 * args.steps,
             "peaks": {"hbm_gbs": hbm, "int8_tops": int8_peak, "source": peaks["source"],
                       "nominal_hbm_gbs": NOMINAL_HBM_GBS, "nominal_int8_tops": NOMINAL_INT8_TOPS},
