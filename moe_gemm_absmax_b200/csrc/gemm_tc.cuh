@@ -112,9 +112,10 @@ struct TcSmem {
     static constexpr int kB = BN * kTcBK;                    // bytes per B stage
     static constexpr int kTiles = STAGES * (kA + kB);
     static constexpr int kBars = (2 * STAGES + 2 * 4 + 1) * 8;
-    // epilogue scratch (group-128 column scales): 8 warps x 64 fp32
+    // epilogue scratch: the group-128 column scales (8 warps x 64 fp32), or
+    // each epilogue warp's copy of the tile's BN column scales
     static constexpr int kEpiOff = kTiles + (kBars + 16 + 15) / 16 * 16;
-    static constexpr int kEpiBytes = 8 * 64 * 4;
+    static constexpr int kEpiBytes = 8 * (BN > 64 ? BN : 64) * 4;
     static constexpr int kBytes = 1024 /*alignment slack*/ + kEpiOff + kEpiBytes;
 };
 
@@ -402,22 +403,42 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                     }
                 }
             } else {
+                // the tile's column scales (per expert in the grouped modes) into this
+                // warp's shared scratch, before the wait: N % 8 == 0, so a 4-column
+                // vector is all in or all out
+                constexpr bool kSw = EPI == kEpiBf16 || EPI == kEpiMoeGated || EPI == kEpiMoeCombine ||
+                                     EPI == kEpiMoeCombineAtomic;
+                float* sw_s = epi_scratch + (warp - 2) * BN;
+                if (kSw) {
+                    __syncwarp();   // the previous tile's reads are done
+                    const float* swt = p.sw + (int64_t)ti.e * p.N;
+                    for (int v = lane; v < BN / 4; v += 32) {
+                        const int n = ti.n0 + 4 * v;
+                        float4 sv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        if (n < p.N) sv = __ldg(reinterpret_cast<const float4*>(swt + n));
+                        *reinterpret_cast<float4*>(sw_s + 4 * v) = sv;
+                    }
+                    __syncwarp();
+                }
                 if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, (kKernelIdGemmTc << 16) | 6)) break;
                 tc_fence_after();
                 float sxr = 0.0f;
                 if ((EPI == kEpiBf16 || EPI == kEpiMoeGated || EPI == kEpiMoeCombine || EPI == kEpiMoeCombineAtomic) &&
                     row_ok)
                     sxr = __ldg(p.sx + row);
-#pragma unroll 1
-                for (int c = (NEPI == 8 ? 32 * chalf : 0); c < BN; c += (NEPI == 8 ? 64 : 32)) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tq + (uint32_t)(acc * BN + c), r);
-                    tc_wait_ld();
+                int64_t orow_i = 0;
+                float wr = 0.0f;
+                if ((EPI == kEpiMoeCombine || EPI == kEpiMoeCombineAtomic) && row_ok) {
+                    orow_i = EPI == kEpiMoeCombine ? (int64_t)__ldg(p.row_tok + row) * p.topk + __ldg(p.row_slot + row)
+                                                   : (int64_t)__ldg(p.row_tok + row);
+                    wr = __ldg(p.row_w + row);
+                }
+                // one 32-column chunk (the next one's TMEM load is in flight)
+                auto chunk = [&](const uint32_t (&r)[32], int c) {
                     const int n0 = nt * BN + c;
-                    if (!row_ok || n0 >= p.N) continue;
+                    if (!row_ok || n0 >= p.N) return;
                     if (EPI == kEpiMoeGated) {
                         // columns n0 .. n0+31 of expert e: 16 (gate, up) pairs
-                        const float* swe = p.sw + (int64_t)ti.e * p.N + n0;
                         float* arow = p.a_out + (int64_t)row * (p.N / 2) + n0 / 2;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -425,55 +446,45 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 const int j = 8 * q + 2 * i;
-                                const float vg = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), __ldg(swe + j));
+                                const float vg = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), sw_s[c + j]);
                                 const float vu =
-                                    __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sxr), __ldg(swe + j + 1));
+                                    __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sxr), sw_s[c + j + 1]);
                                 av[i] = __fmul_rn(silu_proj(vg), vu);
                             }
                             *reinterpret_cast<float4*>(arow + 4 * q) = make_float4(av[0], av[1], av[2], av[3]);
                         }
-                        continue;
-                    }
-                    if (EPI == kEpiMoeCombine || EPI == kEpiMoeCombineAtomic) {
-                        const float* swe = p.sw + (int64_t)ti.e * p.N + n0;
-                        constexpr bool at_slot = EPI == kEpiMoeCombine;
-                        const int64_t orow_i = at_slot
-                                                   ? (int64_t)__ldg(p.row_tok + row) * p.topk + __ldg(p.row_slot + row)
-                                                   : (int64_t)__ldg(p.row_tok + row);
+                    } else if (EPI == kEpiMoeCombine || EPI == kEpiMoeCombineAtomic) {
                         float* orow = p.contrib + orow_i * p.N + n0;
-                        const float wr = __ldg(p.row_w + row);
+                        const uint64_t sx2 = f2_pack(sxr, sxr), w2v = f2_pack(wr, wr);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            float cv[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int j = 4 * q + i;
-                                const float y2 = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sxr), __ldg(swe + j));
-                                cv[i] = __fmul_rn(wr, y2);
-                            }
-                            if constexpr (at_slot)
-                                __stcs(reinterpret_cast<float4*>(orow + 4 * q), make_float4(cv[0], cv[1], cv[2], cv[3]));
+                            const float4 s4 = *reinterpret_cast<const float4*>(sw_s + c + 4 * q);
+                            const uint64_t a01 = f2_pack(__int2float_rn((int)r[4 * q]), __int2float_rn((int)r[4 * q + 1]));
+                            const uint64_t a23 =
+                                f2_pack(__int2float_rn((int)r[4 * q + 2]), __int2float_rn((int)r[4 * q + 3]));
+                            float c0, c1, c2, c3;
+                            f2_unpack(f2_mul(w2v, f2_mul(f2_mul(a01, sx2), f2_pack(s4.x, s4.y))), c0, c1);
+                            f2_unpack(f2_mul(w2v, f2_mul(f2_mul(a23, sx2), f2_pack(s4.z, s4.w))), c2, c3);
+                            if constexpr (EPI == kEpiMoeCombine)
+                                __stcs(reinterpret_cast<float4*>(orow + 4 * q), make_float4(c0, c1, c2, c3));
                             else
-                                red_add_v4(orow + 4 * q, cv[0], cv[1], cv[2], cv[3]);
+                                red_add_v4(orow + 4 * q, c0, c1, c2, c3);
                         }
-                        continue;
-                    }
-                    if (EPI == kEpiBf16) {
+                    } else if (EPI == kEpiBf16) {
                         uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
-                        const float4* swv = reinterpret_cast<const float4*>(p.sw + n0);
+                        const uint64_t sx2 = f2_pack(sxr, sxr);
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {           // 8 columns per 16-byte store
                             if (n0 + v * 8 < p.N) {
-                                const float4 s0 = __ldg(swv + 2 * v);
-                                const float4 s1 = __ldg(swv + 2 * v + 1);
-                                const float sw8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
                                 uint32_t pk[4];
 #pragma unroll
                                 for (int j = 0; j < 4; ++j) {
-                                    const float lo = __fmul_rn(
-                                        __fmul_rn(__int2float_rn((int)r[v * 8 + 2 * j]), sxr), sw8[2 * j]);
-                                    const float hi = __fmul_rn(
-                                        __fmul_rn(__int2float_rn((int)r[v * 8 + 2 * j + 1]), sxr), sw8[2 * j + 1]);
+                                    const uint64_t a2 = f2_pack(__int2float_rn((int)r[v * 8 + 2 * j]),
+                                                                __int2float_rn((int)r[v * 8 + 2 * j + 1]));
+                                    float lo, hi;
+                                    f2_unpack(f2_mul(f2_mul(a2, sx2), f2_pack(sw_s[c + v * 8 + 2 * j],
+                                                                              sw_s[c + v * 8 + 2 * j + 1])),
+                                              lo, hi);
                                     pk[j] = pack_bf16x2(lo, hi);
                                 }
                                 *reinterpret_cast<uint4*>(yrow + n0 + v * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -488,6 +499,22 @@ __global__ void __launch_bounds__(tc_threads<NEPI>(), 1)
                                     make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                         }
                     }
+                };
+                constexpr int kStep = NEPI == 8 ? 64 : 32;
+                uint32_t ra[32], rb[32];
+                int c = NEPI == 8 ? 32 * chalf : 0;
+                const uint32_t tqa = tq + (uint32_t)(acc * BN);
+                if (c < BN) tmem_ld_32x32b_x32(tqa + (uint32_t)c, ra);
+                while (c < BN) {
+                    tc_wait_ld();
+                    if (c + kStep < BN) tmem_ld_32x32b_x32(tqa + (uint32_t)(c + kStep), rb);
+                    chunk(ra, c);
+                    c += kStep;
+                    if (c >= BN) break;
+                    tc_wait_ld();
+                    if (c + kStep < BN) tmem_ld_32x32b_x32(tqa + (uint32_t)(c + kStep), ra);
+                    chunk(rb, c);
+                    c += kStep;
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
