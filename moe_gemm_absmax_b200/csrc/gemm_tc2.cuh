@@ -38,13 +38,13 @@ constexpr int kTc2Epi = 8;        // epilogue warps: TMEM lane quarter x alterna
 constexpr int kTc2Threads = 64 + 32 * kTc2Epi;
 constexpr int kKernelIdGemmTc2 = 4;
 
-// BN columns per pair tile: each CTA holds BN / 2 rows of B (256 or 160).
+// BN columns per pair tile: each CTA holds BN / 2 rows of B (256, 160 or 144).
 // As many stages as fit: at a few hundred tokens every pair streams its own
 // weight columns from HBM, and the bytes in flight per SM set the pace.
 template <int BN>
 struct Tc2Smem {
     static constexpr int kA = 128 * kTcBK;                   // 16 KB per stage
-    static constexpr int kB = (BN / 2) * kTcBK;              // 16 / 10 KB per stage (multiples of 1 KB)
+    static constexpr int kB = (BN / 2) * kTcBK;              // 16 / 10 / 9 KB per stage (multiples of 1 KB)
     static constexpr int kStages = BN == 256 ? 6 : 8;
     static constexpr int kTiles = kStages * (kA + kB);
     static constexpr int kBars = (2 * kStages + 2 + 2 + 1) * 8;
@@ -124,7 +124,7 @@ template <int EPI, int BN = 256>
 __global__ void __launch_bounds__(kTc2Threads, 1)
     gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
     static_assert(EPI == kEpiBf16 || EPI == kEpiS32 || EPI == kEpiMoeGated, "dense epilogues");
-    static_assert(BN % 32 == 0 && (BN / 2) % 8 == 0 && BN <= 256, "pair tile width");
+    static_assert(BN % 16 == 0 && (BN / 2) % 8 == 0 && BN <= 256, "pair tile width");
     constexpr int kCols = 2 * BN <= 256 ? 256 : 512;   // two accumulators of BN columns (a power of two)
     using SM = Tc2Smem<BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -285,12 +285,15 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
             auto chunk = [&](const uint32_t (&r)[32], int c) {
                 const int n0 = nt * BN + c;
                 if (!row_ok || n0 >= p.N) return;
+                // the tile's columns in this chunk (BN % 32 == 16: the last chunk holds
+                // 16; its TMEM load reads 16 columns past the tile, which are ignored)
+                const int ncol = BN - c < 32 ? BN - c : 32;
                 if (EPI == kEpiBf16) {
                     uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + (int64_t)row * p.N;
                     const uint64_t sx2 = f2_pack(sxr, sxr);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
-                        if (n0 + v * 8 < p.N) {
+                        if (v * 8 < ncol && n0 + v * 8 < p.N) {
                             const float4 s0 = *reinterpret_cast<const float4*>(sw_s + c + 8 * v);
                             const float4 s1 = *reinterpret_cast<const float4*>(sw_s + c + 8 * v + 4);
                             const float sw8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
@@ -307,10 +310,12 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                         }
                     }
                 } else if (EPI == kEpiMoeGated) {
-                    // columns n0 .. n0+31: 16 (gate, up) pairs -> a[row, n0/2 .. n0/2+15] (N % 32 == 0)
+                    // columns n0 .. n0+31: 16 (gate, up) pairs -> a[row, n0/2 .. n0/2+15]
+                    // (N % 16 == 0 and n0 % 16 == 0: eight columns are all in or all out)
                     float* arow = p.a_out + (int64_t)row * (p.N / 2) + n0 / 2;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
+                        if (8 * q >= ncol || n0 + 8 * q >= p.N) break;
                         float av[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -325,7 +330,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                     int32_t* orow = reinterpret_cast<int32_t*>(p.out) + (int64_t)row * p.N;
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
-                        if (n0 + v * 4 < p.N)
+                        if (v * 4 < ncol && n0 + v * 4 < p.N)
                             *reinterpret_cast<uint4*>(orow + n0 + v * 4) =
                                 make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                 }

@@ -151,7 +151,7 @@ int launch_tc2_bn(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st)
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, p));
 }
 
-// Pair-tile width: 256 columns, or 160 where the narrower tile's better
+// Pair-tile width: 256 columns, or 160 / 144 where a narrower tile's better
 // filled last wave outweighs its higher operand ingest per MAC.  Per 128-byte
 // k block a CTA spends about max(MMA, ingest) cycles: MMA ~2.78 cycles per
 // column (256 x BN x 128 int8 MACs over the pair), ingest (16 KB of A +
@@ -164,7 +164,10 @@ int pick_tc2_bn(int64_t M, int64_t N, int clusters) {
         const double kblock = std::max(2.78 * bn, (16384.0 + 64.0 * bn) / 43.0);
         return (double)waves * kblock;
     };
-    return cost(160) < cost(256) ? 160 : 256;
+    int best = 256;
+    for (int bn : {160, 144})
+        if (cost(bn) < cost(best)) best = bn;
+    return best;
 }
 
 // Group-128 GEMM on pair tiles (256 x 128).
@@ -208,8 +211,10 @@ int launch_tc2_g128(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t s
 
 template <int EPI>
 int launch_tc2(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st) {
-    return pick_tc2_bn(p.M, p.N, current_sms() / 2) == 160 ? launch_tc2_bn<EPI, 160>(A, B, p, st)
-                                                           : launch_tc2_bn<EPI, 256>(A, B, p, st);
+    const int bn = pick_tc2_bn(p.M, p.N, current_sms() / 2);
+    return bn == 160 ? launch_tc2_bn<EPI, 160>(A, B, p, st)
+         : bn == 144 ? launch_tc2_bn<EPI, 144>(A, B, p, st)
+                     : launch_tc2_bn<EPI, 256>(A, B, p, st);
 }
 
 // Tile width: the one with less work in its last wave (256 on ties).
