@@ -127,10 +127,15 @@ __device__ __forceinline__ void ms_epi_sync() { asm volatile("bar.sync 1, %0;" :
 // Named barrier of one epilogue group of 4 warps (ids 1 and 2).
 __device__ __forceinline__ void ms_group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
-// Threads: producer warp, MMA warp, then 8 epilogue warps (two groups of four
-// for the per-token form, lane quarter x column half for the group-128 form).
+// Threads: weight producer warp, MMA warp, 8 epilogue warps (two groups of
+// four for the per-token form, lane quarter x column half for the group-128
+// form), then the token-code producer warp.  Each k block takes one weight
+// box and one code box; an issuing thread completes about one box per ~340
+// cycles whatever its size, so with both on one thread a CTA would stream
+// its 16 KB weight boxes at about half the rate one thread reaches alone.
+constexpr int kMsXWarp = 10;
 template <bool G128>
-constexpr int ms_threads() { return 320; }
+constexpr int ms_threads() { return 352; }
 
 template <int BN, bool GATED, bool G128 = false>
 __global__ void __launch_bounds__(ms_threads<G128>(), 1)
@@ -203,9 +208,15 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    if (warp == 0) {
-        // ---------------------------------------------------------- producer
+    if (warp == 0 || warp == kMsXWarp) {
+        // ---------------------------------------------------------- producers
+        // warp 0: weight boxes (arming full[s] with the stage's bytes; the first
+        // `pre` stages were armed and started before the wait above); warp
+        // kMsXWarp: the token codes of the same stages.  A code box that lands
+        // before its stage is armed only takes the barrier's transaction count
+        // below zero while the arrival is still pending.
         if (lane == 0) {
+            const bool codes = warp == kMsXWarp;
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_phase = 0;
             int64_t i = 0;   // stage count of this CTA
@@ -220,10 +231,12 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&full[stage], (uint32_t)SM::kStage);
-                        tma_load_2d(smem + stage * SM::kStage, &tmW, &full[stage], kb * kMsBK, wrow);
+                        if (!codes) {
+                            mbar_arrive_expect_tx(&full[stage], (uint32_t)SM::kStage);
+                            tma_load_2d(smem + stage * SM::kStage, &tmW, &full[stage], kb * kMsBK, wrow);
+                        }
                     }
-                    tma_load_2d(smem + stage * SM::kStage + SM::kW, &tmX, &full[stage], kb * kMsBK, k.row0);
+                    if (codes) tma_load_2d(smem + stage * SM::kStage + SM::kW, &tmX, &full[stage], kb * kMsBK, k.row0);
                     issued |= 1u << stage;
                     last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
