@@ -152,10 +152,12 @@ int launch_tc2_bn(const int8_t* A, const int8_t* B, TcParams p, cudaStream_t st)
 }
 
 // Pair-tile width: 256 columns, or 160 / 144 where a narrower tile's better
-// filled last wave outweighs its higher operand ingest per MAC.  Per 128-byte
-// k block a CTA spends about max(MMA, ingest) cycles: MMA ~2.78 cycles per
-// column (256 x BN x 128 int8 MACs over the pair), ingest (16 KB of A +
-// 64 B per column of B) at ~43 B per cycle (both measured on the 256 tile).
+// filled last wave outweighs its higher operand traffic per MAC.  Per 128-byte
+// k block a CTA spends about max(2.78 cycles per column, (16 KB of A + 64 B
+// per column of B) / 43 B per cycle): a fit to the pair kernel's measured
+// rates.  The MMA alone needs 2.0 cycles per column; the 256-wide tile's
+// ~712 cycles come from the SM's shared-memory port, which carries both the
+// TMA writes and the MMA's operand reads.
 int pick_tc2_bn(int64_t M, int64_t N, int clusters) {
     const int64_t mt = (M + kTc2BM - 1) / kTc2BM;
     auto cost = [&](int bn) {
