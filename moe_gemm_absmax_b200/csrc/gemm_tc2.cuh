@@ -43,9 +43,14 @@ constexpr int kKernelIdGemmTc2 = 4;
 // weight columns from HBM, and the bytes in flight per SM set the pace.
 template <int BN>
 struct Tc2Smem {
-    static constexpr int kA = 128 * kTcBK;                   // 16 KB per stage
-    static constexpr int kB = (BN / 2) * kTcBK;              // 16 / 10 / 9 KB per stage (multiples of 1 KB)
-    static constexpr int kStages = BN == 256 ? 6 : 8;
+    // k blocks per stage: the 144 tile (a few hundred tokens, one tile per
+    // cluster) takes two, halving the stage hand-offs per MMA
+    static constexpr int kKB = BN == 144 ? 2 : 1;
+    static constexpr int kA1 = 128 * kTcBK;                  // one k block of A: 16 KB
+    static constexpr int kB1 = (BN / 2) * kTcBK;             // one k block of B: 16 / 10 / 9 KB (multiples of 1 KB)
+    static constexpr int kA = kKB * kA1;
+    static constexpr int kB = kKB * kB1;
+    static constexpr int kStages = BN == 256 ? 6 : (BN == 144 ? 4 : 8);
     static constexpr int kTiles = kStages * (kA + kB);
     static constexpr int kBars = (2 * kStages + 2 + 2 + 1) * 8;
     // each epilogue warp's copy of the tile's column scales (fp32)
@@ -185,15 +190,21 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
             bool ok = true;
             for (int tile = cluster_id; ok && tile < num_tiles; tile += nclusters) {
                 const int mt = tile % p.num_m_tiles, nt = tile / p.num_m_tiles;
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = 0; kb < p.num_k_blocks; kb += SM::kKB) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, (kKernelIdGemmTc2 << 16) | 1)) {
                         ok = false;
                         break;
                     }
                     const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2u * (SM::kA + SM::kB));
-                    tma_load_2d_pair(sA + stage * SM::kA, &tmA, fb, kb * kTcBK, mt * kTc2BM + (int)rank * 128);
-                    tma_load_2d_pair(sB + stage * SM::kB, &tmB, fb, kb * kTcBK, nt * BN + (int)rank * (BN / 2));
+                    // a k block past K (odd count) reads as zeros and adds nothing
+#pragma unroll
+                    for (int j = 0; j < SM::kKB; ++j) {
+                        tma_load_2d_pair(sA + stage * SM::kA + j * SM::kA1, &tmA, fb, (kb + j) * kTcBK,
+                                         mt * kTc2BM + (int)rank * 128);
+                        tma_load_2d_pair(sB + stage * SM::kB + j * SM::kB1, &tmB, fb, (kb + j) * kTcBK,
+                                         nt * BN + (int)rank * (BN / 2));
+                    }
                     issued |= 1u << stage;
                     last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == SM::kStages) {
@@ -223,18 +234,21 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = 0; kb < p.num_k_blocks; kb += SM::kKB) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, (kKernelIdGemmTc2 << 16) | 4)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * SM::kA);
-                    const uint32_t b0 = smem_u32(sB + stage * SM::kB);
 #pragma unroll
-                    for (int kk = 0; kk < kTcBK / 32; ++kk)
-                        tc2_mma_i8(d_tmem, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
-                                   (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int j = 0; j < SM::kKB; ++j) {
+                        const uint32_t a0 = smem_u32(sA + stage * SM::kA + j * SM::kA1);
+                        const uint32_t b0 = smem_u32(sB + stage * SM::kB + j * SM::kB1);
+#pragma unroll
+                        for (int kk = 0; kk < kTcBK / 32; ++kk)
+                            tc2_mma_i8(d_tmem, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32),
+                                       idesc, (kb > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc2_commit_pair(&empty[stage]);   // frees this stage in both CTAs
                     if (++stage == SM::kStages) {
                         stage = 0;
