@@ -49,10 +49,16 @@ constexpr int kMsSlots = 8;         // TMEM accumulators of the group-128 form: 
 
 template <int BN, bool G128 = false>
 struct MsSmem {
-    static constexpr int kStages = BN <= 32 ? 10 : 8;
+    // k blocks per stage: two in the per-token form (its MMAs of N = 16-64
+    // take 262 cycles per k block, too few to cover the ring's per-stage
+    // hand-off); one in the group-128 form (a TMEM slot per k block)
+    static constexpr int kKB = G128 ? 1 : 2;
+    static constexpr int kStages = G128 ? (BN <= 32 ? 10 : 8) : (BN <= 32 ? 5 : 4);
     static constexpr int kNAcc = G128 ? kMsSlots : 2;
-    static constexpr int kW = kMsBM * kMsBK;        // 16 KB
-    static constexpr int kX = BN * kMsBK;           // 2 / 4 / 8 KB
+    static constexpr int kW1 = kMsBM * kMsBK;       // one k block of weights: 16 KB
+    static constexpr int kX1 = BN * kMsBK;          // one k block of codes: 2 / 4 / 8 KB
+    static constexpr int kW = kKB * kW1;
+    static constexpr int kX = kKB * kX1;
     static constexpr int kStage = kW + kX;          // multiple of 1024
     static constexpr int kTiles = kStages * kStage;
     static constexpr int kBars = (2 * kStages + 2 * kNAcc + 1) * 8;
@@ -192,17 +198,21 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
     __syncthreads();
     const int nunits = sp[a.E] * a.ngroups;
     const int my_units = nunits > (int)blockIdx.x ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const int64_t my_stages = (int64_t)my_units * a.nkb;
+    const int nst = (a.nkb + SM::kKB - 1) / SM::kKB;   // stages per unit
+    const int64_t my_stages = (int64_t)my_units * nst;
     const int pre = my_stages < STAGES ? (int)my_stages : STAGES;   // stages armed before the wait
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmW);
         prefetch_tensormap(&tmX);
-        for (int i = 0; i < pre; ++i) {   // unit blockIdx.x + (i / nkb) * gridDim.x, k block i % nkb
-            const int u = blockIdx.x + (i / a.nkb) * gridDim.x;
+        for (int i = 0; i < pre; ++i) {   // unit blockIdx.x + (i / nst) * gridDim.x, k blocks from kKB (i % nst)
+            const int u = blockIdx.x + (i / nst) * gridDim.x;
             const int b = u / a.ngroups, g = u - b * a.ngroups;
             const MsBlock k = ms_block(sp, a.E, b, BN);
             mbar_arrive_expect_tx(&full[i], (uint32_t)SM::kStage);
-            tma_load_2d(smem + i * SM::kStage, &tmW, &full[i], (i % a.nkb) * kMsBK, k.e * a.rows + g * kMsBM);
+#pragma unroll
+            for (int j = 0; j < SM::kKB; ++j)   // a k block past K (odd count) reads as zeros
+                tma_load_2d(smem + i * SM::kStage + j * SM::kW1, &tmW, &full[i], ((i % nst) * SM::kKB + j) * kMsBK,
+                            k.e * a.rows + g * kMsBM);
         }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -225,7 +235,7 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                 const int b = u / a.ngroups, g = u - b * a.ngroups;
                 const MsBlock k = ms_block(sp, a.E, b, BN);
                 const int wrow = k.e * a.rows + g * kMsBM;
-                for (int kb = 0; kb < a.nkb; ++kb, ++i) {
+                for (int kb = 0; kb < a.nkb; kb += SM::kKB, ++i) {
                     if (i >= pre) {
                         if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, (kKernelIdMoeSwap << 16) | 1)) {
                             ok = false;
@@ -233,10 +243,18 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                         }
                         if (!codes) {
                             mbar_arrive_expect_tx(&full[stage], (uint32_t)SM::kStage);
-                            tma_load_2d(smem + stage * SM::kStage, &tmW, &full[stage], kb * kMsBK, wrow);
+#pragma unroll
+                            for (int j = 0; j < SM::kKB; ++j)
+                                tma_load_2d(smem + stage * SM::kStage + j * SM::kW1, &tmW, &full[stage],
+                                            (kb + j) * kMsBK, wrow);
                         }
                     }
-                    if (codes) tma_load_2d(smem + stage * SM::kStage + SM::kW, &tmX, &full[stage], kb * kMsBK, k.row0);
+                    if (codes) {
+#pragma unroll
+                        for (int j = 0; j < SM::kKB; ++j)
+                            tma_load_2d(smem + stage * SM::kStage + SM::kW + j * SM::kX1, &tmX, &full[stage],
+                                        (kb + j) * kMsBK, k.row0);
+                    }
                     issued |= 1u << stage;
                     last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -313,18 +331,21 @@ __global__ void __launch_bounds__(ms_threads<G128>(), 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < a.nkb; ++kb) {
+                for (int kb = 0; kb < a.nkb; kb += SM::kKB) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, (kKernelIdMoeSwap << 16) | 4)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t w0 = smem_u32(smem + stage * SM::kStage);
-                    const uint32_t x0 = w0 + SM::kW;
 #pragma unroll
-                    for (int kk = 0; kk < kMsBK / 32; ++kk)
-                        tc_mma_i8(d_tmem, smem_desc_k_sw128(w0 + kk * 32), smem_desc_k_sw128(x0 + kk * 32), idesc,
-                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int j = 0; j < SM::kKB; ++j) {
+                        const uint32_t w0 = smem_u32(smem + stage * SM::kStage + j * SM::kW1);
+                        const uint32_t x0 = smem_u32(smem + stage * SM::kStage + SM::kW + j * SM::kX1);
+#pragma unroll
+                        for (int kk = 0; kk < kMsBK / 32; ++kk)
+                            tc_mma_i8(d_tmem, smem_desc_k_sw128(w0 + kk * 32), smem_desc_k_sw128(x0 + kk * 32),
+                                      idesc, (kb > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
