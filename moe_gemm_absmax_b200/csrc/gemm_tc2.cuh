@@ -39,8 +39,10 @@ constexpr int kTc2Threads = 64 + 32 * kTc2Epi;
 constexpr int kKernelIdGemmTc2 = 4;
 
 // BN columns per pair tile: each CTA holds BN / 2 rows of B (256, 160 or 144).
-// As many stages as fit: at a few hundred tokens every pair streams its own
-// weight columns from HBM, and the bytes in flight per SM set the pace.
+// As many stages as fit.  A stage carries enough MMA work to cover the ring's
+// per-stage hand-off (MMA completion -> empty -> producer -> full -> MMA
+// thread): one k block for the 256 and 160 tiles (512 / 320 cycles of MMA),
+// two for the 144 tile (2 x 288).
 template <int BN>
 struct Tc2Smem {
     // k blocks per stage: the 144 tile (a few hundred tokens, one tile per

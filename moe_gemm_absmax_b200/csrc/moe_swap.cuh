@@ -42,7 +42,7 @@
 namespace w8a8 {
 
 constexpr int kMsBM = 128;          // weight rows per group (MMA M)
-constexpr int kMsBK = 128;          // bytes of K per stage
+constexpr int kMsBK = 128;          // bytes of K per k block (a ring stage holds one or two)
 constexpr int kKernelIdMoeSwap = 5;
 constexpr int kMsMaxGroups = 32;    // K / 128 of the group-128 form
 constexpr int kMsSlots = 8;         // TMEM accumulators of the group-128 form: one per k block in flight
