@@ -113,6 +113,20 @@ def test_linear_prefill_m512_every_output(orc, shape):
     assert np.array_equal(y, yo)
 
 
+def test_linear_pair_tile_odd_k_blocks(orc):
+    """The 144-column pair tile (chosen for N = 5120 at M = 512) loads two
+    128-byte k blocks per ring stage; with K = 17280 (135 k blocks) its last
+    stage's second block lies past K and must add nothing.  Every output."""
+    M, N, K = 512, 5120, 17280
+    rng = np.random.default_rng(17)
+    xb = inputs.dense_linear(41, M, K, 16, with_weights=False)[0]
+    qw, sw = orc.quant_rows_f32(inputs.weights(rng, (N, K)))
+    y = from_dev_bf16(w8a8.linear(to_dev_bf16(xb), torch.from_numpy(qw).cuda(), torch.from_numpy(sw).cuda()))
+    yo, y32, _, _ = orc.linear(xb, qw, sw)
+    assert assert_bf16_close(y, y32, what="pair tile, odd k blocks") == 1.0
+    assert np.array_equal(y, yo)
+
+
 def test_linear_prefill_ragged_rows(orc):
     xb, qw, sw = _quantized(orc, 5, 300, 1024, 776)
     y = w8a8.linear(to_dev_bf16(xb), torch.from_numpy(qw).cuda(), torch.from_numpy(sw).cuda())
